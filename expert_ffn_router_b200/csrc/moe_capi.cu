@@ -1,0 +1,468 @@
+// The C ABI of libmoe: argument validation, workspace carving and the launch
+// sequence of each entry point.  Every step of the layer runs in this
+// library's kernels; the host only checks arguments and enqueues launches.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+#include "moe.h"
+#include "moe_launch.h"
+#include "moe_route.cuh"
+
+namespace moe {
+
+static thread_local std::string g_last_error;
+
+static moe_status fail(moe_status st, const std::string& msg) {
+    g_last_error = msg;
+    return st;
+}
+
+static moe_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(MOE_ECUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------------------
+// cached device facts
+// ---------------------------------------------------------------------------
+static std::mutex g_mu;
+static std::unordered_map<unsigned long long, int> g_grid;  // (device, func, smem) -> grid
+static std::unordered_map<unsigned long long, size_t> g_smem;
+
+static unsigned long long cache_key(int dev, const void* func, size_t smem) {
+    return ((unsigned long long)(uintptr_t)func * 1000003ull) ^ ((unsigned long long)smem << 20) ^
+           (unsigned long long)dev;
+}
+
+int persistent_grid(const void* func, size_t smem) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long key = cache_key(dev, func, smem);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_grid.find(key);
+        if (it != g_grid.end()) return it->second;
+    }
+    int sms = 0, per_sm = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, kThreads, smem);
+    const int grid = std::max(1, sms * std::max(1, per_sm));
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_grid[key] = grid;
+    return grid;
+}
+
+cudaError_t allow_smem(const void* func, size_t smem) {
+    if (smem <= 48 * 1024) return cudaSuccess;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long key = cache_key(dev, func, 0);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_smem.find(key);
+        if (it != g_smem.end() && it->second >= smem) return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_smem[key] = smem;
+    }
+    return e;
+}
+
+static int round_ncl(int ncl, bool down) {
+    if (ncl <= 1) return 1;
+    if (ncl <= 2) return 2;
+    if (ncl <= 4) return 4;
+    if (!down && ncl <= 6) return 6;
+    return 8;
+}
+
+ExpertTiling expert_tiling(int d, int f, int wb) {
+    ExpertTiling t{};
+    const int nch3 = d * wb / 8 / 16, nch4 = f * wb / 8 / 16;
+    t.ncl3 = round_ncl((nch3 + 31) / 32, false);
+    t.rpw3 = rpw3();
+    t.ncl4 = round_ncl((nch4 + 31) / 32, true);
+    t.rpw4 = rpw4(t.ncl4);
+    return t;
+}
+
+// ---------------------------------------------------------------------------
+// validation
+// ---------------------------------------------------------------------------
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static moe_status check_cfg(const moe_config* c) {
+    if (!c) return fail(MOE_EINVAL, "cfg is NULL");
+    if (c->d <= 0 || c->f <= 0 || c->d > 8192 || c->f > 8192)
+        return fail(MOE_EINVAL, "d and f must be in [1, 8192]");
+    if (c->wbits != 4 && c->wbits != 2) return fail(MOE_EINVAL, "wbits must be 4 or 2");
+    if ((c->d * c->wbits / 8) % 16 || (c->f * c->wbits / 8) % 16 || (c->d * c->wbits) % 8 || (c->f * c->wbits) % 8)
+        return fail(MOE_EINVAL, "d*wbits/8 and f*wbits/8 must be multiples of 16 bytes");
+    if (c->n_experts < 1 || c->n_experts > 1024) return fail(MOE_EINVAL, "n_experts must be in [1, 1024]");
+    if (c->top_k < 1 || c->top_k > 32 || c->top_k > c->n_experts)
+        return fail(MOE_EINVAL, "top_k must be in [1, min(n_experts, 32)]");
+    if (c->has_shared != 0 && c->has_shared != 1) return fail(MOE_EINVAL, "has_shared must be 0 or 1");
+    if (!(c->routed_scale == c->routed_scale)) return fail(MOE_EINVAL, "routed_scale is NaN");
+    return MOE_OK;
+}
+
+static moe_status check_ptr(const void* p, const char* name, bool nullable = false) {
+    if (!p) return nullable ? MOE_OK : fail(MOE_EINVAL, std::string(name) + " is NULL");
+    if (!aligned16(p)) return fail(MOE_EALIGN, std::string(name) + " is not 16-byte aligned");
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                       \
+    do {                                    \
+        moe_status _st = (expr);            \
+        if (_st != MOE_OK) return _st;      \
+    } while (0)
+
+static Dims dims_of(const moe_config* c, int T, int S) {
+    return Dims{c->d, c->f, c->n_experts, c->top_k, c->has_shared, c->wbits, T, S};
+}
+
+static int pick_ch(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8; }
+
+static Params base_params(const moe_config* c, const Dims& m, void* ws) {
+    Params p{};
+    p.m = m;
+    p.routed_scale = c->routed_scale;
+    p.blob_bytes = 3ll * c->d * c->f * c->wbits / 8;
+    p.scale_rows = 2 * c->f + c->d;
+    p.CH = pick_ch(m.T);
+    const ExpertTiling tl = expert_tiling(c->d, c->f, c->wbits);
+    p.rb3 = kWarps * tl.rpw3;
+    p.nrb3 = (c->f + p.rb3 - 1) / p.rb3;
+    p.rb4 = kWarps * tl.rpw4;
+    p.nrb4 = (c->d + p.rb4 - 1) / p.rb4;
+    p.ksplit = 1;
+    p.ws = ws_carve(m, ws);
+    return p;
+}
+
+static moe_status check_ws(const Dims& m, void* ws, size_t ws_bytes) {
+    MOE_TRY(check_ptr(ws, "ws"));
+    const size_t need = ws_carve(m, nullptr).bytes;
+    if (ws_bytes < need)
+        return fail(MOE_ENOSPACE, "workspace has " + std::to_string(ws_bytes) + " bytes, needs " + std::to_string(need));
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// router launch sequence (a0 + a1 (+ a2))
+// ---------------------------------------------------------------------------
+template <int TM, typename XT>
+static cudaError_t route_small_nv(Params& p, const XT* x, int do_quant, int bucket, cudaStream_t s) {
+    const int E = p.m.E;
+    const size_t smem = std::max((size_t)2 * kWarps * E * 4, (size_t)(4 * E + kWarps) * 4);
+    const int nv = p.m.d / 4;
+    const int per = (nv + kThreads - 1) / kThreads;
+    const int grid = (E + 1) / 2;
+#define MOE_RS(NV)                                                                   \
+    {                                                                                \
+        auto fn = k_route_small<TM, NV, XT>;                                         \
+        cudaError_t e = allow_smem((const void*)fn, smem);                           \
+        if (e != cudaSuccess) return e;                                              \
+        fn<<<grid, kThreads, smem, s>>>(p, x, do_quant, bucket);                     \
+        return cudaGetLastError();                                                   \
+    }
+    if (per <= 2) MOE_RS(2)
+    if (per <= 6) MOE_RS(6)
+    MOE_RS(8)
+#undef MOE_RS
+}
+
+template <typename XT>
+static cudaError_t launch_router(Params& p, const XT* x, int do_quant, int bucket, cudaStream_t s) {
+    const int T = p.m.T, E = p.m.E, d = p.m.d;
+    if (T <= 8) {
+        p.ksplit = 1;
+        switch (T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8) {
+            case 1: return route_small_nv<1>(p, x, do_quant, bucket, s);
+            case 2: return route_small_nv<2>(p, x, do_quant, bucket, s);
+            case 4: return route_small_nv<4>(p, x, do_quant, bucket, s);
+            default: return route_small_nv<8>(p, x, do_quant, bucket, s);
+        }
+    }
+    cudaError_t e;
+    if (do_quant) {
+        k_quantize<XT><<<std::min(T, 65535), kThreads, 0, s>>>(x, T, d, p.ws.xq, p.ws.sx, p.ws.xcs);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // split d so that the tiled GEMM fills the GPU (slices of whole 32-column steps)
+    const int tiles = ((E + 63) / 64) * ((T + 63) / 64);
+    const int ksteps = d / 32;
+    int ks = std::max(1, std::min(std::min(ksteps, kRouterKsplitMax), (2 * 148 + tiles - 1) / tiles));
+    const int per = (ksteps + ks - 1) / ks;
+    ks = (ksteps + per - 1) / per;
+    p.ksplit = ks;
+    k_router_tiled<XT><<<dim3((E + 63) / 64, (T + 63) / 64, ks), kThreads, 0, s>>>(p, x);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t smem_topk = (size_t)2 * kWarps * E * 4;
+    if ((e = allow_smem((const void*)k_topk, smem_topk)) != cudaSuccess) return e;
+    k_topk<<<(T + kWarps - 1) / kWarps, kThreads, smem_topk, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (bucket) {
+        k_bucket<<<1, kThreads, (size_t)(4 * E + kWarps) * 4, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+static cudaError_t launch_router_any(Params& p, const void* x, moe_dtype dt, int do_quant, int bucket,
+                                     cudaStream_t s) {
+    if (dt == MOE_BF16) return launch_router(p, static_cast<const __nv_bfloat16*>(x), do_quant, bucket, s);
+    return launch_router(p, static_cast<const float*>(x), do_quant, bucket, s);
+}
+
+static moe_status check_dtype(moe_dtype dt) {
+    return (dt == MOE_F32 || dt == MOE_BF16) ? MOE_OK : fail(MOE_EINVAL, "dtype must be MOE_F32 or MOE_BF16");
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_config* cfg, int32_t max_tokens) {
+    if (check_cfg(cfg) != MOE_OK || max_tokens < 0) return 0;
+    const int S = cfg->top_k + cfg->has_shared;
+    return ws_carve(dims_of(cfg, std::max(1, (int)max_tokens), S), nullptr).bytes;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_TRY(check_ptr(ws, "ws"));
+    if (ws_bytes < sizeof(WsHeader)) return fail(MOE_ENOSPACE, "workspace smaller than its header");
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_workspace_init");
+}
+
+moe_status moe_quantize(const moe_config* cfg, const void* x, moe_dtype dtype, int32_t T, int8_t* xq, float* sx,
+                        moe_stream_t stream) {
+    MOE_TRY(check_cfg(cfg));
+    MOE_TRY(check_dtype(dtype));
+    if (T < 0) return fail(MOE_EINVAL, "T < 0");
+    if (T == 0) return MOE_OK;
+    MOE_TRY(check_ptr(x, "x"));
+    MOE_TRY(check_ptr(xq, "xq"));
+    MOE_TRY(check_ptr(sx, "sx"));
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = std::min((int)T, 65535);
+    if (dtype == MOE_BF16)
+        k_quantize<__nv_bfloat16><<<grid, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, cfg->d, xq, sx,
+                                                             nullptr);
+    else
+        k_quantize<float><<<grid, kThreads, 0, s>>>(static_cast<const float*>(x), T, cfg->d, xq, sx, nullptr);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_quantize");
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, moe_dtype dtype, int32_t T, const float* w_router,
+                     const float* bias, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                     moe_stream_t stream) {
+    MOE_TRY(check_cfg(cfg));
+    MOE_TRY(check_dtype(dtype));
+    if (T < 0) return fail(MOE_EINVAL, "T < 0");
+    if (T == 0) return MOE_OK;
+    MOE_TRY(check_ptr(x, "x"));
+    MOE_TRY(check_ptr(w_router, "w_router"));
+    MOE_TRY(check_ptr(bias, "bias"));
+    MOE_TRY(check_ptr(topk_idx, "topk_idx"));
+    MOE_TRY(check_ptr(topk_w, "topk_w"));
+    const Dims m = dims_of(cfg, T, cfg->top_k + cfg->has_shared);
+    MOE_TRY(check_ws(m, ws, ws_bytes));
+    Params p = base_params(cfg, m, ws);
+    p.w_router = w_router;
+    p.bias = bias;
+    p.idx_out = topk_idx;
+    p.w_out = topk_w;
+    cudaError_t e = launch_router_any(p, x, dtype, 0, 0, (cudaStream_t)stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route");
+}
+
+static moe_status expert_common(const moe_config* cfg, const moe_pool* pool, int32_t expert, int32_t T, float* y,
+                                void* ws, size_t ws_bytes, Params* out_p) {
+    MOE_TRY(check_cfg(cfg));
+    if (!pool) return fail(MOE_EINVAL, "pool is NULL");
+    MOE_TRY(check_ptr(pool->w, "pool->w"));
+    MOE_TRY(check_ptr(pool->s, "pool->s"));
+    if (T < 0) return fail(MOE_EINVAL, "T < 0");
+    if (expert < -1 || expert >= cfg->n_experts) return fail(MOE_EINVAL, "expert out of range");
+    if (expert == -1 && !cfg->has_shared) return fail(MOE_EINVAL, "no shared expert in this config");
+    MOE_TRY(check_ptr(y, "y"));
+    const Dims m = dims_of(cfg, T, 1);
+    MOE_TRY(check_ws(m, ws, ws_bytes));
+    Params p = base_params(cfg, m, ws);
+    p.pool = pool->w;
+    p.scales = pool->s;
+    p.direct_out = 1;
+    p.out = y;
+    *out_p = p;
+    return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const moe_pool* pool, int32_t expert, const int8_t* xq,
+                          const float* sx, int32_t T, float* y, int32_t* dbg_acc_gu, int8_t* dbg_hq, float* dbg_sh,
+                          int32_t* dbg_acc_d, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Params p;
+    MOE_TRY(expert_common(cfg, pool, expert, T, y, ws, ws_bytes, &p));
+    if (T == 0) return MOE_OK;
+    MOE_TRY(check_ptr(xq, "xq"));
+    MOE_TRY(check_ptr(sx, "sx"));
+    MOE_TRY(check_ptr(dbg_acc_gu, "dbg_acc_gu", true));
+    MOE_TRY(check_ptr(dbg_hq, "dbg_hq", true));
+    MOE_TRY(check_ptr(dbg_sh, "dbg_sh", true));
+    MOE_TRY(check_ptr(dbg_acc_d, "dbg_acc_d", true));
+    const bool dbg = dbg_acc_gu || dbg_hq || dbg_sh || dbg_acc_d;
+    if (dbg) p.CH = 8;
+    p.dbg_acc_gu = dbg_acc_gu;
+    p.dbg_hq = dbg_hq;
+    p.dbg_sh = dbg_sh;
+    p.dbg_acc_d = dbg_acc_d;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int blob = expert < 0 ? cfg->n_experts : expert;
+    // the expert kernels read the activations from the workspace: copy them in
+    cudaError_t e = cudaMemcpyAsync(p.ws.xq, xq, (size_t)T * cfg->d, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(p.ws.sx, sx, (size_t)T * 4, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn copy");
+    k_sum_codes<<<std::min((int)T, 65535), kThreads, 0, s>>>(p.ws.xq, T, cfg->d, p.ws.xcs);
+    k_plan_single<<<1, kThreads, 0, s>>>(p, blob);
+    const ExpertTiling tl = expert_tiling(cfg->d, cfg->f, cfg->wbits);
+    if ((e = cudaGetLastError()) == cudaSuccess) e = launch_gate_up(p, tl, dbg, s);
+    if (e == cudaSuccess) e = launch_down(p, tl, dbg, s);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn");
+}
+
+moe_status moe_expert_down(const moe_config* cfg, const moe_pool* pool, int32_t expert, const int8_t* hq,
+                           const float* sh, int32_t T, float* y, int32_t* dbg_acc_d, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+    Params p;
+    MOE_TRY(expert_common(cfg, pool, expert, T, y, ws, ws_bytes, &p));
+    if (T == 0) return MOE_OK;
+    MOE_TRY(check_ptr(hq, "hq"));
+    MOE_TRY(check_ptr(sh, "sh"));
+    MOE_TRY(check_ptr(dbg_acc_d, "dbg_acc_d", true));
+    const bool dbg = dbg_acc_d != nullptr;
+    if (dbg) p.CH = 8;
+    p.hq_in = hq;
+    p.sh_in = sh;
+    p.dbg_acc_d = dbg_acc_d;
+    cudaStream_t s = (cudaStream_t)stream;
+    k_plan_single<<<1, kThreads, 0, s>>>(p, expert < 0 ? cfg->n_experts : expert);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = launch_down(p, expert_tiling(cfg->d, cfg->f, cfg->wbits), dbg, s);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_down");
+}
+
+moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float* w_router, const float* bias,
+                        const void* x, moe_dtype dtype, int32_t T, float* out, int32_t accumulate,
+                        int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                        moe_layer_opts* opts) {
+    MOE_TRY(check_cfg(cfg));
+    MOE_TRY(check_dtype(dtype));
+    if (!pool) return fail(MOE_EINVAL, "pool is NULL");
+    if (T < 0) return fail(MOE_EINVAL, "T < 0");
+    if (opts) opts->n_launches = 0;
+    if (T == 0) return MOE_OK;
+    MOE_TRY(check_ptr(pool->w, "pool->w"));
+    MOE_TRY(check_ptr(pool->s, "pool->s"));
+    MOE_TRY(check_ptr(w_router, "w_router"));
+    MOE_TRY(check_ptr(bias, "bias"));
+    MOE_TRY(check_ptr(x, "x"));
+    MOE_TRY(check_ptr(out, "out"));
+    MOE_TRY(check_ptr(topk_idx_out, "topk_idx_out", true));
+    MOE_TRY(check_ptr(topk_w_out, "topk_w_out", true));
+    const Dims m = dims_of(cfg, T, cfg->top_k + cfg->has_shared);
+    MOE_TRY(check_ws(m, ws, ws_bytes));
+    Params p = base_params(cfg, m, ws);
+    p.pool = pool->w;
+    p.scales = pool->s;
+    p.w_router = w_router;
+    p.bias = bias;
+    p.out = out;
+    p.accumulate = accumulate ? 1 : 0;
+    p.idx_out = topk_idx_out;
+    p.w_out = topk_w_out;
+    cudaStream_t s = (cudaStream_t)stream;
+    const ExpertTiling tl = expert_tiling(cfg->d, cfg->f, cfg->wbits);
+    auto mark = [&](int i) -> cudaError_t {
+        if (opts && opts->events[i]) return cudaEventRecord((cudaEvent_t)opts->events[i], s);
+        return cudaSuccess;
+    };
+    cudaError_t e = mark(0);
+    if (e == cudaSuccess) e = launch_router_any(p, x, dtype, 1, 1, s);
+    if (e == cudaSuccess) e = mark(1);
+    if (e == cudaSuccess) e = launch_gate_up(p, tl, false, s);
+    if (e == cudaSuccess) e = mark(2);
+    if (e == cudaSuccess) e = launch_down(p, tl, false, s);
+    if (e == cudaSuccess) e = mark(3);
+    if (opts) opts->n_launches = (T <= 8 ? 1 : 4) + 2;
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer");
+}
+
+moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const float* w_router, const float* bias,
+                     const void* x, moe_dtype dtype, int32_t T, float* out, int32_t accumulate, int32_t* topk_idx_out,
+                     float* topk_w_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return moe_layer_ex(cfg, pool, w_router, bias, x, dtype, T, out, accumulate, topk_idx_out, topk_w_out, ws,
+                        ws_bytes, stream, nullptr);
+}
+
+moe_status moe_rmsnorm(const void* x, moe_dtype dtype, int32_t T, int32_t d, float eps, float* x_in, float* x_copy,
+                       moe_stream_t stream) {
+    MOE_TRY(check_dtype(dtype));
+    if (T < 0 || d <= 0 || d % 4) return fail(MOE_EINVAL, "T >= 0 and d > 0, a multiple of 4, required");
+    if (T == 0) return MOE_OK;
+    MOE_TRY(check_ptr(x, "x"));
+    MOE_TRY(check_ptr(x_in, "x_in"));
+    MOE_TRY(check_ptr(x_copy, "x_copy", true));
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = std::min((int)T, 65535);
+    if (dtype == MOE_BF16)
+        k_rmsnorm<__nv_bfloat16><<<grid, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, d, eps, x_in,
+                                                           x_copy);
+    else
+        k_rmsnorm<float><<<grid, kThreads, 0, s>>>(static_cast<const float*>(x), T, d, eps, x_in, x_copy);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_rmsnorm");
+}
+
+moe_status moe_poll_status(const void* ws, int32_t* info, moe_stream_t stream) {
+    MOE_TRY(check_ptr(ws, "ws"));
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_poll_status sync");
+    int32_t hv[2] = {0, 0};
+    e = cudaMemcpy(hv, ws, sizeof(hv), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_poll_status copy");
+    if (info) *info = hv[1];
+    if (hv[0] != 0) return fail((moe_status)hv[0], "a kernel reported an error (info " + std::to_string(hv[1]) + ")");
+    return MOE_OK;
+}
+
+const char* moe_status_string(moe_status st) {
+    switch (st) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_EINVAL: return "MOE_EINVAL: invalid argument";
+        case MOE_EALIGN: return "MOE_EALIGN: pointer not 16-byte aligned";
+        case MOE_ENOSPACE: return "MOE_ENOSPACE: workspace too small";
+        case MOE_ECUDA: return "MOE_ECUDA: CUDA error";
+        case MOE_ETIMEOUT: return "MOE_ETIMEOUT: bounded device wait expired";
+        case MOE_EDEVICE: return "MOE_EDEVICE: a kernel found an invalid value";
+        default: return "unknown moe_status";
+    }
+}
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,370 @@
+// Shared device/host helpers of libmoe: workspace layout, kernel parameters,
+// PTX wrappers, block reductions and the int8 activation staging layout.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kThreads = 256;  // every kernel of the library runs 256-thread CTAs
+constexpr int kWarps = kThreads / 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// Workspace: a 256-byte header of control words followed by the per-call
+// buffers.  Offsets depend on (cfg, T) only, so any workspace of at least
+// moe_workspace_bytes(cfg, T) bytes serves a call with T tokens.
+// ---------------------------------------------------------------------------
+struct WsHeader {
+    int32_t status;       // first error code a kernel reported (0 = none)
+    int32_t status_info;  // detail word of that error
+    uint32_t route_ctr;   // arrival ticket of the router CTAs (self-resetting)
+    int32_t n_tasks;      // tasks = (expert, <= CH tokens) pairs of this call
+    int32_t n_asg;        // assignments incl. shared-expert ones
+    int32_t n_items3;     // gate/up work items
+    int32_t n_items4;     // down work items
+    int32_t pad[57];
+};
+static_assert(sizeof(WsHeader) == 256, "header must stay 256 bytes");
+
+struct Ws {
+    WsHeader* hdr;
+    int8_t* xq;        // [T][d]     quantised activations
+    float* sx;         // [T]        activation scales
+    int32_t* xcs;      // [T]        sum of each token's codes
+    float* logits;     // [ksplit][T][E] router logits (partials when split over d)
+    int32_t* idx;      // [T][k]     routing
+    float* w;          // [T][k]     routing weights
+    int32_t* asg;      // [T*S]      assignment ids (token*S + slot) grouped by task
+    int4* tasks;       // [max_tasks] (blob, asg start, n tokens, 0)
+    uint32_t* task_ctr;// [max_tasks] gate/up item arrivals per task (self-resetting)
+    uint32_t* amax;    // [T*S]      max |h| per assignment (float bits)
+    float* h;          // [T*S][f]   SwiGLU output
+    int8_t* hq;        // [T*S][f]   requantised h
+    float* sh;         // [T*S]      scale of hq
+    float* ybuf;       // [T*S][d]   per-assignment down outputs before the combine
+    uint32_t* rb_ctr;  // [ceil(d/rb4)] down item arrivals per row block (self-resetting)
+    size_t bytes;
+};
+
+constexpr int kRouterKsplitMax = 64;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Dims {
+    int d, f, E, k, has_shared, wb, T, S;
+};
+
+inline int max_tasks(const Dims& m) { return m.T * m.S + m.E + 2; }
+// Rows per warp per work item of the gate/up and down kernels (one definition
+// for the kernels' template arguments and the host's item counts).
+constexpr int rpw3() { return 2; }
+constexpr int rpw4(int ncl) { return ncl >= 8 ? 1 : 8 / ncl; }
+constexpr int kMinRowBlock4 = 8;  // smallest down row block: 8 warps x rpw4(8)
+
+inline Ws ws_carve(const Dims& m, void* base) {
+    Ws w{};
+    char* b = static_cast<char*>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> void* {
+        void* p = b ? b + off : nullptr;
+        off = align_up(off + bytes, 256);
+        return p;
+    };
+    const size_t T = (size_t)m.T, A = (size_t)m.T * m.S;
+    w.hdr = (WsHeader*)take(sizeof(WsHeader));
+    w.xq = (int8_t*)take(T * m.d);
+    w.sx = (float*)take(T * 4);
+    w.xcs = (int32_t*)take(T * 4);
+    w.logits = (float*)take((size_t)kRouterKsplitMax * T * m.E * 4);
+    w.idx = (int32_t*)take(T * m.k * 4);
+    w.w = (float*)take(T * m.k * 4);
+    w.asg = (int32_t*)take(A * 4);
+    w.tasks = (int4*)take((size_t)max_tasks(m) * 16);
+    w.task_ctr = (uint32_t*)take((size_t)max_tasks(m) * 4);
+    w.amax = (uint32_t*)take(A * 4);
+    w.h = (float*)take(A * m.f * 4);
+    w.hq = (int8_t*)take(A * m.f);
+    w.sh = (float*)take(A * 4);
+    w.ybuf = (float*)take(A * m.d * 4);
+    w.rb_ctr = (uint32_t*)take((size_t)((m.d + kMinRowBlock4 - 1) / kMinRowBlock4) * 4);
+    w.bytes = off;
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel parameters (passed by value).
+// ---------------------------------------------------------------------------
+struct Params {
+    Dims m;
+    float routed_scale;
+    const uint8_t* pool;
+    const float* scales;
+    long long blob_bytes;
+    int scale_rows;
+    int CH;          // max tokens per task
+    int rb3, nrb3;   // gate/up rows per item, items per task
+    int rb4, nrb4;   // down rows per item, items per task
+    int ksplit;      // router split of d
+    Ws ws;
+    const float* w_router;
+    const float* bias;
+    float* out;
+    int accumulate;
+    int32_t* idx_out;
+    float* w_out;
+    // single-expert entry points
+    int direct_out;        // write y[token][d] instead of the slot buffer + combine
+    const int8_t* hq_in;   // teacher-forced down: given codes [T][f]
+    const float* sh_in;    // and scales [T]
+    // debug outputs
+    int32_t* dbg_acc_gu;
+    int8_t* dbg_hq;
+    float* dbg_sh;
+    int32_t* dbg_acc_d;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+// Streaming 16-byte load of read-only weights: no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float4 ld_stream_f4(const void* p) {
+    float4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+        : "l"(p));
+    return v;
+}
+// unsigned 8-bit x signed 8-bit 4-way dot product accumulate
+__device__ __forceinline__ int dp4a_us(unsigned a, int b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+__device__ __forceinline__ void set_status(WsHeader* h, int code, int info) {
+    if (atomicCAS(&h->status, 0, code) == 0) atomicExch(&h->status_info, info);
+}
+
+// ---------------------------------------------------------------------------
+// Reductions for 256-thread CTAs
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+// Block reductions; `red` is a kWarps-element shared scratch the caller owns.
+__device__ __forceinline__ float block_max(float v, float* red) {
+    v = warp_max(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int i = 1; i < kWarps; ++i) r = fmaxf(r, red[i]);
+    return r;
+}
+__device__ __forceinline__ float block_sum(float v, float* red) {
+    v = warp_sum(v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int i = 1; i < kWarps; ++i) r += red[i];
+    return r;
+}
+__device__ __forceinline__ int block_sum_int(int v, int* red) {
+    v = __reduce_add_sync(kFull, v);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int r = 0;
+#pragma unroll
+    for (int i = 0; i < kWarps; ++i) r += red[i];
+    return r;
+}
+
+// In-place exclusive scan of n <= 4 * 256 ints in shared memory by a 256-thread
+// CTA; returns the total.  `red` is kWarps ints of shared scratch.
+static __device__ int block_exscan(int* a, int n, int* red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (n + kThreads - 1) / kThreads;
+    const int b = tid * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i)
+        if (b + i < n) local += a[b + i];
+    int v = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += y;
+    }
+    __syncthreads();
+    if (lane == 31) red[warp] = v;
+    __syncthreads();
+    int base = 0, total = 0;
+#pragma unroll
+    for (int i = 0; i < kWarps; ++i) {
+        if (i < warp) base += red[i];
+        total += red[i];
+    }
+    int run = base + v - local;
+    for (int i = 0; i < per; ++i)
+        if (b + i < n) {
+            int t = a[b + i];
+            a[b + i] = run;
+            run += t;
+        }
+    __syncthreads();
+    return total;
+}
+
+// ---------------------------------------------------------------------------
+// Activation staging layout.  A 16-byte chunk of packed weights holds 32 int4
+// codes (or 64 int2 codes).  The dot kernels split each weight word into
+// byte lanes with one mask (offset-binary codes u = c + 8 or c + 2), so the
+// int8 activations are stored per chunk in the matching byte order:
+//  int4: per 8 columns, word E = (x0,x2,x4,x6) then word O = (x1,x3,x5,x7);
+//        sub-array s (s = 0, 1) of a chunk holds columns 16s .. 16s+15.
+//  int2: per 16 columns, words P_m = (x_m, x_{m+4}, x_{m+8}, x_{m+12}),
+//        m = 0..3; sub-array s (s = 0..3) holds columns 16s .. 16s+15.
+// Shared-memory layout of one staged row: [NSUB][nch] uint4, nch = chunks per
+// row, NSUB = 8 / wbits, so a warp reading consecutive chunks is conflict-free.
+// ---------------------------------------------------------------------------
+template <int WB>
+__device__ __forceinline__ uint4 permute16(uint4 n) {
+    uint4 r;
+    if (WB == 4) {
+        r.x = __byte_perm(n.x, n.y, 0x6420);
+        r.y = __byte_perm(n.x, n.y, 0x7531);
+        r.z = __byte_perm(n.z, n.w, 0x6420);
+        r.w = __byte_perm(n.z, n.w, 0x7531);
+    } else {
+        unsigned a_lo = __byte_perm(n.x, n.y, 0x5140), b_lo = __byte_perm(n.z, n.w, 0x5140);
+        unsigned a_hi = __byte_perm(n.x, n.y, 0x7362), b_hi = __byte_perm(n.z, n.w, 0x7362);
+        r.x = __byte_perm(a_lo, b_lo, 0x5410);
+        r.y = __byte_perm(a_lo, b_lo, 0x7632);
+        r.z = __byte_perm(a_hi, b_hi, 0x5410);
+        r.w = __byte_perm(a_hi, b_hi, 0x7632);
+    }
+    return r;
+}
+
+// Sum of the 16 signed bytes of a uint4.
+__device__ __forceinline__ int sum16(uint4 v) {
+    int s = 0;
+    s = __dp4a((int)v.x, 0x01010101, s);
+    s = __dp4a((int)v.y, 0x01010101, s);
+    s = __dp4a((int)v.z, 0x01010101, s);
+    s = __dp4a((int)v.w, 0x01010101, s);
+    return s;
+}
+
+// Stage one int8 row of `ncols` codes (global, 16-byte aligned) into the
+// permuted layout at `dst` ([NSUB][nch] uint4); returns this thread's partial
+// sum of the codes (the caller reduces it).
+template <int WB>
+__device__ __forceinline__ int stage_row(const int8_t* src, int ncols, uint4* dst) {
+    constexpr int NSUB = 8 / WB;
+    const int n16 = ncols / 16;          // 16-byte pieces
+    const int nch = n16 / NSUB;          // weight chunks per row
+    int s = 0;
+    for (int i = threadIdx.x; i < n16; i += kThreads) {
+        uint4 v = __ldcg(reinterpret_cast<const uint4*>(src) + i);
+        s += sum16(v);
+        const int c = i / NSUB, sub = i % NSUB;
+        dst[sub * nch + c] = permute16<WB>(v);
+    }
+    return s;
+}
+
+// Dot of one 16-byte weight chunk with one staged activation chunk.
+template <int WB>
+__device__ __forceinline__ int dot_chunk(const uint4 w, const uint4* xs, int nch, int c, int acc) {
+    if (WB == 4) {
+        const uint4 x0 = xs[c], x1 = xs[nch + c];
+        const unsigned a = w.x ^ 0x88888888u, b = w.y ^ 0x88888888u;
+        const unsigned cc = w.z ^ 0x88888888u, dd = w.w ^ 0x88888888u;
+        acc = dp4a_us(a & 0x0F0F0F0Fu, (int)x0.x, acc);
+        acc = dp4a_us((a >> 4) & 0x0F0F0F0Fu, (int)x0.y, acc);
+        acc = dp4a_us(b & 0x0F0F0F0Fu, (int)x0.z, acc);
+        acc = dp4a_us((b >> 4) & 0x0F0F0F0Fu, (int)x0.w, acc);
+        acc = dp4a_us(cc & 0x0F0F0F0Fu, (int)x1.x, acc);
+        acc = dp4a_us((cc >> 4) & 0x0F0F0F0Fu, (int)x1.y, acc);
+        acc = dp4a_us(dd & 0x0F0F0F0Fu, (int)x1.z, acc);
+        acc = dp4a_us((dd >> 4) & 0x0F0F0F0Fu, (int)x1.w, acc);
+    } else {
+        const unsigned ws[4] = {w.x ^ 0xAAAAAAAAu, w.y ^ 0xAAAAAAAAu, w.z ^ 0xAAAAAAAAu, w.w ^ 0xAAAAAAAAu};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const uint4 xv = xs[s * nch + c];
+            acc = dp4a_us(ws[s] & 0x03030303u, (int)xv.x, acc);
+            acc = dp4a_us((ws[s] >> 2) & 0x03030303u, (int)xv.y, acc);
+            acc = dp4a_us((ws[s] >> 4) & 0x03030303u, (int)xv.z, acc);
+            acc = dp4a_us((ws[s] >> 6) & 0x03030303u, (int)xv.w, acc);
+        }
+    }
+    return acc;
+}
+
+// Offset of the offset-binary codes: sum c*x = sum u*x - kOff * sum x.
+template <int WB>
+__device__ __forceinline__ constexpr int code_offset() { return WB == 4 ? 8 : 2; }
+
+// Quantiser rule of the layer (fp32, IEEE division, round half to even).
+__device__ __forceinline__ int quant_code(float v, float s) {
+    int q = __float2int_rn(__fdiv_rn(v, s));
+    return max(-127, min(127, q));
+}
+
+template <typename XT>
+__device__ __forceinline__ float load_x(const XT* x, size_t i);
+template <>
+__device__ __forceinline__ float load_x<float>(const float* x, size_t i) { return __ldg(x + i); }
+template <>
+__device__ __forceinline__ float load_x<__nv_bfloat16>(const __nv_bfloat16* x, size_t i) {
+    return __bfloat162float(x[i]);
+}
+
+// 4 consecutive activations (i multiple of 4) as float4.
+template <typename XT>
+__device__ __forceinline__ float4 load_x4(const XT* x, size_t i);
+template <>
+__device__ __forceinline__ float4 load_x4<float>(const float* x, size_t i) {
+    return __ldg(reinterpret_cast<const float4*>(x + i));
+}
+template <>
+__device__ __forceinline__ float4 load_x4<__nv_bfloat16>(const __nv_bfloat16* x, size_t i) {
+    uint2 v = __ldg(reinterpret_cast<const uint2*>(x + i));
+    float4 r;
+    r.x = __uint_as_float(v.x << 16);
+    r.y = __uint_as_float(v.x & 0xFFFF0000u);
+    r.z = __uint_as_float(v.y << 16);
+    r.w = __uint_as_float(v.y & 0xFFFF0000u);
+    return r;
+}
+
+}  // namespace moe

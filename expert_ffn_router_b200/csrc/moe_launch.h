@@ -1,0 +1,26 @@
+// Internal launchers shared by the translation units of libmoe (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+// Tiling choices of the expert kernels for a given shape.
+struct ExpertTiling {
+    int ncl3, rpw3;  // gate/up: 16-byte chunks per lane per row, rows per warp per item
+    int ncl4, rpw4;  // down: the same
+};
+
+ExpertTiling expert_tiling(int d, int f, int wb);
+
+// Persistent-grid size for a kernel: SMs x resident CTAs (cached per kernel).
+int persistent_grid(const void* func, size_t smem);
+// Raise the dynamic shared-memory limit of a kernel once (cached).
+cudaError_t allow_smem(const void* func, size_t smem);
+
+cudaError_t launch_gate_up(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s);
+cudaError_t launch_down(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,180 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed-expert MoE layer library, libmoe.so.
+ *
+ * The layer is the one the Colibri pages describe for streaming-MoE inference
+ * of GLM-5.2 (744B): a DeepSeek-V3-style router picks top-k of E routed
+ * experts per token (takumi3488 article, teacher-forcing section; top-8 of 256
+ * in the coli info log), every expert is a feed-forward block whose weights are
+ * packed int4 or int2 codes with per-row scales, dequantised on use and
+ * multiplied against int8 activations with integer dot products (agentlenshq
+ * summary, "Integer-Dot Kernels" and "Quantization"), and the routed outputs
+ * are combined with the always-resident shared expert (agentlenshq summary,
+ * "Memory split").  An expert requested by several tokens of a batch is read
+ * once (remio.ai analysis, the paragraph on merging duplicate expert requests).
+ *
+ * Conventions for every call:
+ *  - Tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or keeps caller memory beyond the stream work it
+ *    enqueues.  Pointers must be 16-byte aligned (MOE_EALIGN otherwise).
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) with no implicit synchronisation.  Argument errors are detected
+ *    on the host before anything is enqueued and return synchronously.  A
+ *    failed launch returns MOE_ECUDA.  Errors found by the kernels themselves
+ *    are written to a status word in the workspace; read it with
+ *    moe_poll_status after synchronising the stream.
+ *  - The library keeps no global handles and is safe to call from several
+ *    host threads; calls that share one workspace must not overlap on the GPU.
+ *  - moe_last_error() returns a thread-local description of the last failure.
+ *
+ * Numerics (identical on every entry point):
+ *  - activation quantiser: per token s = max|x| / 127 (fp32, IEEE division),
+ *    code = clamp(round_half_even(x / s), -127, 127); an all-zero token gets
+ *    s = 0 and zero codes; bf16 inputs are widened exactly to fp32 first.
+ *  - router: logits = W_r x in fp32 on the UNQUANTISED x; score = sigmoid;
+ *    selection on score + bias, descending, ties to the lower expert index;
+ *    weights = selected scores / their sum * routed_scale (bias not included).
+ *  - codes: two's complement, low bits first (int4 byte = c0 | c1 << 4; int2
+ *    byte = c0 | c1 << 2 | c2 << 4 | c3 << 6); int32 accumulation is exact.
+ *  - gate/up: g = acc_g * (s_row * s_x), u likewise, h = g / (1 + exp(-g)) * u
+ *    (SwiGLU); h is requantised per (token, expert) with the activation rule.
+ *  - down: y = acc_d * (s_row * s_h); out = sum_j w_j y_j + y_shared (fp32).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_EINVAL = -1,   /* bad dimension, null pointer or unsupported combination   */
+    MOE_EALIGN = -2,   /* a pointer is not 16-byte aligned                          */
+    MOE_ENOSPACE = -3, /* workspace smaller than moe_workspace_bytes(cfg, T)        */
+    MOE_ECUDA = -4,    /* a CUDA runtime call or kernel launch failed               */
+    MOE_ETIMEOUT = -5, /* a bounded device-side wait ran out (status word only)     */
+    MOE_EDEVICE = -6   /* a kernel found an invalid value, e.g. an index out of range */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Shape of one MoE layer.
+ *  d: hidden size; f: expert intermediate size; n_experts: routed experts E;
+ *  top_k: experts per token k; has_shared: 1 if a shared expert follows the E
+ *  routed blobs; wbits: 4 or 2; routed_scale: factor on the renormalised
+ *  routed weights (2.5 for GLM-5.2).
+ *  tc_min_tokens: experts with at least this many tokens in a call run on the
+ *  int8 tensor-core (tcgen05) path; 0 = library default, < 0 = never.
+ * Limits (MOE_EINVAL otherwise): 1 <= k <= min(E, 32); E <= 1024;
+ * d * wbits / 8 and f * wbits / 8 multiples of 16; d <= 8192; f <= 8192. */
+typedef struct {
+    int32_t d, f, n_experts, top_k, has_shared, wbits;
+    float routed_scale;
+    int32_t tc_min_tokens;
+} moe_config;
+
+/* One layer's experts, resident in device memory, canonical layout.
+ *  w: E + has_shared blobs of 3*d*f*wbits/8 bytes each, expert e at offset
+ *     e * blob_bytes, the shared expert last.  A blob is
+ *     [gate f x d | up f x d | down d x f], each matrix row-major by output
+ *     row, codes packed as above ("adjacent matrices stored together").
+ *  s: fp32 [E + has_shared][f + f + d] per-output-row scales, same order. */
+typedef struct {
+    const uint8_t* w;
+    const float* s;
+} moe_pool;
+
+/* Bytes of workspace the calls below need for up to max_tokens tokens. */
+MOE_API size_t moe_workspace_bytes(const moe_config* cfg, int32_t max_tokens);
+
+/* Zero the workspace control words.  Call once after allocating a workspace
+ * (and after a call that reported a device error) before its first use; the
+ * kernels leave the control words at zero between calls. */
+MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Activation quantiser alone (step a0), exposed for parity checks.
+ * x [T][d] (dtype) -> xq int8 [T][d], sx fp32 [T]. */
+MOE_API moe_status moe_quantize(const moe_config* cfg, const void* x, moe_dtype dtype, int32_t T, int8_t* xq,
+                        float* sx, moe_stream_t stream);
+
+/* Router alone (step a1): x [T][d] (dtype), w_router fp32 [E][d], bias fp32
+ * [E] -> topk_idx int32 [T][k] (slot order = selection score descending),
+ * topk_w fp32 [T][k]. */
+MOE_API moe_status moe_route(const moe_config* cfg, const void* x, moe_dtype dtype, int32_t T,
+                     const float* w_router, const float* bias, int32_t* topk_idx, float* topk_w,
+                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* One expert over T tokens (steps a3 + a4): expert in [0, E) is a routed
+ * expert, -1 the shared one.  xq int8 [T][d], sx fp32 [T] -> y fp32 [T][d]
+ * (overwritten).  Optional debug outputs (NULL to skip): dbg_acc_gu int32
+ * [T][2f] (gate accumulators then up accumulators), dbg_hq int8 [T][f],
+ * dbg_sh fp32 [T], dbg_acc_d int32 [T][d]. */
+MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const moe_pool* pool, int32_t expert, const int8_t* xq,
+                          const float* sx, int32_t T, float* y, int32_t* dbg_acc_gu, int8_t* dbg_hq,
+                          float* dbg_sh, int32_t* dbg_acc_d, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/* Down projection alone from given h codes (step a4, for teacher-forced
+ * parity): hq int8 [T][f], sh fp32 [T] -> y fp32 [T][d]; dbg_acc_d optional. */
+MOE_API moe_status moe_expert_down(const moe_config* cfg, const moe_pool* pool, int32_t expert, const int8_t* hq,
+                           const float* sh, int32_t T, float* y, int32_t* dbg_acc_d, void* ws,
+                           size_t ws_bytes, moe_stream_t stream);
+
+/* The whole layer (steps a0-a7): quantise, route, bucket tokens by expert
+ * (each selected expert is read once per call), gate/up, requantise, down,
+ * weighted combine with the shared expert.
+ * x [T][d] (dtype) -> out fp32 [T][d]: overwritten if accumulate == 0, added
+ * to if accumulate != 0 (residual stream of stacked layers).  topk_idx_out
+ * int32 [T][k] and topk_w_out fp32 [T][k] are optional copies of the routing. */
+MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const float* w_router, const float* bias,
+                     const void* x, moe_dtype dtype, int32_t T, float* out, int32_t accumulate,
+                     int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/* Options of moe_layer_ex (all optional; zero-initialise).
+ *  events: cudaEvent_t handles (or NULL) recorded on `stream` before routing
+ *          [0], after routing and bucketing [1], after gate/up [2] and after
+ *          down + combine [3]; for timing the phases on the launching stream.
+ *  n_launches: set to the number of kernels the call launched. */
+typedef struct {
+    void* events[4];
+    int32_t n_launches;
+    int32_t reserved[7];
+} moe_layer_opts;
+
+/* moe_layer with options (opts may be NULL, then identical to moe_layer). */
+MOE_API moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float* w_router,
+                                const float* bias, const void* x, moe_dtype dtype, int32_t T, float* out,
+                                int32_t accumulate, int32_t* topk_idx_out, float* topk_w_out, void* ws,
+                                size_t ws_bytes, moe_stream_t stream, moe_layer_opts* opts);
+
+/* Parameter-free RMSNorm of a residual stream, used between stacked layers:
+ * x_in = x / sqrt(mean(x^2) + eps).  x [T][d] (dtype) -> x_in fp32 [T][d].
+ * If x_copy is not NULL it receives x widened to fp32 (to start a residual
+ * stream from bf16 activations). */
+MOE_API moe_status moe_rmsnorm(const void* x, moe_dtype dtype, int32_t T, int32_t d, float eps, float* x_in,
+                       float* x_copy, moe_stream_t stream);
+
+/* Device-side status word of a workspace (MOE_OK if no kernel reported an
+ * error).  Synchronises `stream` first.  *info (optional) receives a detail
+ * word. */
+MOE_API moe_status moe_poll_status(const void* ws, int32_t* info, moe_stream_t stream);
+
+MOE_API const char* moe_status_string(moe_status status);
+MOE_API const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,268 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs, through the C ABI.
+
+Small shapes span several row blocks, a ragged lane tail (16-byte chunks per
+row not a multiple of 32) and both router paths (GEMV for T <= 8, tiled for
+larger T); full shapes are the decode, MTP-verify, prefill and skewed int2
+workloads, checked on every token the oracle can afford (all of them for the
+decode-sized ones, a sample for prefill and the 24-layer stack).
+"""
+import numpy as np
+import pytest
+import torch
+
+import expert_ffn_router_b200 as M
+import oracle as O
+import workloads as W
+from parity_utils import HQ_MAX_FRAC, OUT_REL_L2, hq_close, rel_l2, routing_mismatches
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": W.workload(0),
+    "ragged_int4": W.workload(0).replace(name="ragged_int4", d=1056, f=352, n_experts=40, top_k=6, T=37),
+    "ragged_int4_T5": W.workload(0).replace(name="ragged_int4", d=1056, f=352, n_experts=40, top_k=6, T=5),
+    "ragged_int2": W.workload(0).replace(name="ragged_int2", d=1088, f=320, n_experts=24, top_k=5, T=13, wbits=2),
+    "k_eq_E": W.workload(0).replace(name="k_eq_E", d=256, f=128, n_experts=4, top_k=4, T=9),
+    "no_shared": W.workload(0).replace(name="no_shared", d=512, f=256, n_experts=16, top_k=3, T=3,
+                                       has_shared=0),
+}
+
+
+def cfg_of(wl):
+    return M.config(wl.d, wl.f, wl.n_experts, wl.top_k, wl.has_shared, wl.wbits, wl.routed_scale)
+
+
+def x_host(wl, token_set=0, T=None):
+    return W.tokens(wl, 0, token_set, T)
+
+
+def to_dev(t):
+    return t.contiguous().cuda()
+
+
+def assert_ok(ws):
+    assert M.moe_poll_status(ws) == M.MOE_OK
+
+
+@pytest.mark.parametrize("name", list(SMALL) + ["bf16_d6144"])
+def test_quantize_bitexact(name):
+    wl = SMALL.get(name) or W.workload(1)
+    x = x_host(wl, 3, 64 if name == "bf16_d6144" else None)
+    x[1].zero_()  # an all-zero token
+    q_o, s_o = O.quantize(x.float())
+    xq = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    sx = torch.empty(x.shape[0], dtype=torch.float32, device="cuda")
+    M.moe_quantize(cfg_of(wl), to_dev(x), xq, sx)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(xq.cpu().numpy(), q_o)
+    np.testing.assert_array_equal(sx.cpu().numpy(), s_o)
+
+
+def check_route(wl, x, L, report):
+    cfg = cfg_of(wl)
+    T = x.shape[0]
+    idx = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, wl.top_k, dtype=torch.float32, device="cuda")
+    ws = M.workspace(cfg, T)
+    M.moe_route(cfg, to_dev(x), to_dev(L.w_router), to_dev(L.bias), idx, w, ws)
+    assert_ok(ws)
+    o_idx, o_w, _, _, o_sel = O.route(x.float(), L.w_router, L.bias, wl.top_k, wl.routed_scale, want_scores=True)
+    g_idx = idx.cpu().numpy()
+    allowed, bad = routing_mismatches(g_idx, o_idx, o_sel)
+    assert bad == [], f"routing differs beyond the near-tie rule on tokens {bad}"
+    report.append((wl.name, T, len(allowed)))
+    keep = [t for t in range(T) if t not in allowed]
+    np.testing.assert_allclose(w.cpu().numpy()[keep], o_w[keep], rtol=2e-6, atol=1e-7)
+    return g_idx
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_route_small(name):
+    wl = SMALL[name]
+    rep = []
+    check_route(wl, x_host(wl), W.layer(wl, 0, 0), rep)
+
+
+@pytest.mark.parametrize("T", [1, 4, 8, 64, 512])
+def test_route_full_size(T):
+    wl = W.workload(4 if T == 64 else 1)
+    rep = []
+    check_route(wl, x_host(wl, 1, T), W.layer(wl, 0, 0), rep)
+    print("near-tie routing mismatches:", rep)
+
+
+EXPERT_CASES = [("tiny", 4, 1), ("ragged_int4", 9, 1), ("ragged_int4", 3, -1), ("ragged_int2", 11, 2),
+                ("full_int4", 1, 7), ("full_int4", 9, -1), ("full_int2", 3, 5)]
+
+
+@pytest.mark.parametrize("name,T,expert", EXPERT_CASES)
+def test_expert_stages(name, T, expert):
+    if name.startswith("full"):
+        wl = W.workload(1 if name == "full_int4" else 4)
+    else:
+        wl = SMALL[name]
+    cfg = cfg_of(wl)
+    e = wl.n_experts if expert < 0 else expert
+    blob = W.expert_blob(wl, 0, 0, e)
+    sc = W.expert_scales(wl, 0, 0, e)
+    # a device pool holding only this expert's blob at its slot (others zero)
+    pool_w = torch.zeros(wl.pool_bytes, dtype=torch.uint8, device="cuda")
+    pool_w[e * wl.blob_bytes:(e + 1) * wl.blob_bytes] = blob.cuda()
+    pool_s = torch.zeros(wl.n_blobs, wl.scale_rows, dtype=torch.float32, device="cuda")
+    pool_s[e] = sc.cuda()
+    pool = M.make_pool(pool_w, pool_s)
+    x = x_host(wl, 2, T).float()
+    xq_o, sx_o = O.quantize(x)
+    r = O.expert(wl.d, wl.f, wl.wbits, blob, sc, xq_o, sx_o)
+    ws = M.workspace(cfg, T)
+    y = torch.empty(T, wl.d, device="cuda")
+    acc_gu = torch.empty(T, 2 * wl.f, dtype=torch.int32, device="cuda")
+    hq = torch.empty(T, wl.f, dtype=torch.int8, device="cuda")
+    sh = torch.empty(T, device="cuda")
+    acc_d = torch.empty(T, wl.d, dtype=torch.int32, device="cuda")
+    M.moe_expert_ffn(cfg, pool, expert, torch.from_numpy(xq_o).cuda(), torch.from_numpy(sx_o).cuda(), y, ws,
+                     acc_gu, hq, sh, acc_d)
+    assert_ok(ws)
+    np.testing.assert_array_equal(acc_gu.cpu().numpy(), r["acc_gu"])
+    mx, frac = hq_close(hq.cpu().numpy(), r["hq"])
+    assert mx <= 1 and frac <= HQ_MAX_FRAC, (mx, frac)
+    np.testing.assert_allclose(sh.cpu().numpy(), r["sh"], rtol=1e-6)
+    # teacher-forced down on the oracle's codes: bit-exact accumulators
+    y2 = torch.empty(T, wl.d, device="cuda")
+    acc_d2 = torch.empty(T, wl.d, dtype=torch.int32, device="cuda")
+    M.moe_expert_down(cfg, pool, expert, torch.from_numpy(r["hq"]).cuda(), torch.from_numpy(r["sh"]).cuda(), y2, ws,
+                      acc_d2)
+    assert_ok(ws)
+    np.testing.assert_array_equal(acc_d2.cpu().numpy(), r["acc_d"])
+    np.testing.assert_allclose(y2.cpu().numpy(), r["y"], rtol=1e-6, atol=1e-30)
+    # the fused path's output against the oracle's
+    assert rel_l2(y.cpu().numpy(), r["y"]) <= OUT_REL_L2
+
+
+def run_layer_gpu(wl, dl, x, accumulate_into=None):
+    cfg = cfg_of(wl)
+    T = x.shape[0]
+    pool = M.make_pool(dl.pool_w, dl.pool_s)
+    out = accumulate_into if accumulate_into is not None else torch.empty(T, wl.d, device="cuda")
+    idx = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, wl.top_k, device="cuda")
+    ws = M.workspace(cfg, T)
+    M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x), out, ws, accumulate=accumulate_into is not None,
+                topk_idx_out=idx, topk_w_out=w)
+    assert_ok(ws)
+    return out, idx.cpu().numpy(), w.cpu().numpy()
+
+
+def compare_layer(wl, L, x, out, g_idx, tokens=None):
+    xf = x.float()
+    if tokens is not None:
+        xf = xf[tokens]
+        out = out[tokens]
+        g_idx = g_idx[tokens]
+    r = O.workload_layer(wl, 0, 0, xf, L=L)
+    _, _, _, _, o_sel = O.route(xf, L.w_router, L.bias, wl.top_k, wl.routed_scale, want_scores=True)
+    allowed, bad = routing_mismatches(g_idx, r["idx"], o_sel)
+    assert bad == [], bad
+    keep = [t for t in range(xf.shape[0]) if t not in allowed]
+    err = rel_l2(out.cpu().numpy()[keep], r["out"][keep])
+    assert err <= OUT_REL_L2, err
+    return err, allowed
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_small(name):
+    wl = SMALL[name]
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    x = x_host(wl)
+    out, g_idx, _ = run_layer_gpu(wl, dl, x)
+    compare_layer(wl, L, x, out, g_idx)
+    # accumulate mode adds the layer to what is there
+    base = torch.randn(x.shape[0], wl.d, device="cuda")
+    acc, _, _ = run_layer_gpu(wl, dl, x, accumulate_into=base.clone())
+    np.testing.assert_allclose(acc.cpu().numpy(), (base + out).cpu().numpy(), rtol=1e-6, atol=1e-5)
+
+
+def test_layer_decode_full_size():
+    """The decode workload as the bench runs it: T = 1 per call, 8 token sets."""
+    wl = W.workload(1)
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    errs = []
+    for s in range(8):
+        x = x_host(wl, s)
+        out, g_idx, _ = run_layer_gpu(wl, dl, x)
+        err, allowed = compare_layer(wl, L, x, out, g_idx)
+        errs.append(err)
+    print("decode rel L2 per token:", errs)
+
+
+def test_layer_prefill_sampled():
+    wl = W.workload(3)
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    x = x_host(wl)
+    out, g_idx, _ = run_layer_gpu(wl, dl, x)
+    tokens = list(range(0, wl.T, 64)) + [wl.T - 1]
+    err, _ = compare_layer(wl, L, x, out, g_idx, tokens)
+    print("prefill sampled rel L2:", err)
+
+
+def run_stack(wl, n_layers, token_subset):
+    """GPU stack over every token; the oracle's own stack over a token subset."""
+    T = wl.T
+    x0 = x_host(wl)
+    resid = torch.empty(T, wl.d, device="cuda")
+    x_in = torch.empty(T, wl.d, device="cuda")
+    M.moe_rmsnorm(to_dev(x0), x_in, 1e-6, x_copy=resid)
+    idxs = []
+    for l in range(n_layers):
+        if l > 0:
+            M.moe_rmsnorm(resid, x_in, 1e-6)
+        dl = W.device_layer(wl, 0, l)
+        _, g_idx, _ = run_layer_gpu(wl, dl, x_in, accumulate_into=resid)
+        idxs.append(g_idx)
+        del dl
+    torch.cuda.synchronize()
+    r = O.workload_stack(wl, 0, x0[token_subset], n_layers)
+    return resid.cpu().numpy()[token_subset], idxs, r
+
+
+@pytest.mark.parametrize("which,n_layers,tokens", [(2, 8, [0, 1, 2, 3]), (4, 24, [0, 37])])
+def test_stacked_layers(which, n_layers, tokens):
+    wl = W.workload(which)
+    g_x, g_idxs, r = run_stack(wl, n_layers, tokens)
+    diverged = set()
+    for l in range(n_layers):
+        L = W.layer(wl, 0, l)
+        _, _, _, _, sel = O.route(r["x_in"][l], L.w_router, L.bias, wl.top_k, wl.routed_scale, want_scores=True)
+        allowed, bad = routing_mismatches(g_idxs[l][tokens], r["idx"][l], sel)
+        assert bad == [] or set(bad) <= diverged, (l, bad)
+        diverged |= {tokens[i] for i in allowed + bad}
+    keep = [i for i, t in enumerate(tokens) if t not in diverged]
+    assert keep, "every sampled token hit a near-tie"
+    err = rel_l2(g_x[keep], r["x"][keep])
+    print(f"stack {wl.name}: final residual rel L2 {err:.3g}, near-tie tokens {sorted(diverged)}")
+    assert err <= OUT_REL_L2
+
+
+def test_workspace_reuse_and_status():
+    """Back-to-back calls on one workspace stay correct (self-resetting counters)."""
+    wl = SMALL["ragged_int4"]
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    cfg = cfg_of(wl)
+    ws = M.workspace(cfg, wl.T)
+    pool = M.make_pool(dl.pool_w, dl.pool_s)
+    outs = []
+    for T in (wl.T, 1, 5, wl.T):
+        x = to_dev(x_host(wl, T, T))
+        out = torch.empty(T, wl.d, device="cuda")
+        M.moe_layer(cfg, pool, dl.w_router, dl.bias, x, out, ws)
+        outs.append(out)
+    assert M.moe_poll_status(ws) == M.MOE_OK
+    ref = torch.empty_like(outs[0])
+    ws2 = M.workspace(cfg, wl.T)
+    M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x_host(wl, wl.T, wl.T)), ref, ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], ref) and torch.equal(outs[3], ref)  # deterministic

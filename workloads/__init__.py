@@ -281,3 +281,18 @@ class Layer:
 def layer(wl: Workload, seed: int, layer_idx: int) -> Layer:
     return Layer(wl, seed, layer_idx, pool_scales(wl, seed, layer_idx),
                  router_weight(wl, seed, layer_idx), router_bias(wl, seed, layer_idx))
+
+
+@dataclasses.dataclass
+class DeviceLayer:
+    """One layer's inputs resident on a device (pool bytes generated there)."""
+    pool_w: torch.Tensor    # uint8 [n_blobs * blob_bytes]
+    pool_s: torch.Tensor    # fp32 [n_blobs][2f+d]
+    w_router: torch.Tensor  # fp32 [E][d]
+    bias: torch.Tensor      # fp32 [E]
+
+
+def device_layer(wl: Workload, seed: int, layer_idx: int, device="cuda", host: Optional[Layer] = None) -> DeviceLayer:
+    L = host if host is not None else layer(wl, seed, layer_idx)
+    w = pool_bytes(wl, seed, layer_idx, device=device)
+    return DeviceLayer(w, L.scales.to(device), L.w_router.to(device), L.bias.to(device))
