@@ -36,13 +36,15 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=1, help="workload id (1 = decode T=1, the metric's config)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--n-experts", type=int, default=0,
+                    help="profiling case: the same layer with fewer routed experts (smaller pool)")
     return ap.parse_args()
 
 
@@ -77,6 +79,11 @@ class Clocks:
         except Exception:
             self.proc = None
         return self
+
+    def wait_first(self, timeout=10.0):
+        t0 = time.time()
+        while self.proc is not None and not self.rows and time.time() - t0 < timeout:
+            time.sleep(0.02)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -209,6 +216,14 @@ def gpu_arm(args, wl):
     idx = torch.empty(T, wl.top_k, dtype=torch.int32, device=dev)
     ws = M.workspace(cfg, T, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(256 << 18, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2(i):
+        # write 256 MiB (evicts the step's lines), then read another 256 MiB so
+        # the dirty lines are written back here, not inside the next timed step
+        flush.fill_(i & 0xFF)
+        torch.sum(flush_rd, dim=0, out=sink)
     stream = torch.cuda.current_stream()
     n_ev = K
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_ev)]
@@ -228,15 +243,16 @@ def gpu_arm(args, wl):
         M.moe_layer(cfg, pool, dl.w_router, dl.bias, xbuf, out, ws, topk_idx_out=log, opts=o)
 
     for i in range(Wm):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         step(i)
     assert M.moe_poll_status(ws) == M.MOE_OK
     barrier()
     torch.cuda.synchronize()
     launches = 0
     with Clocks(local) as clk:
+        clk.wait_first()
         for i in range(K):
-            flush.fill_(i & 0xFF)
+            flush_l2(i)
             xbuf.copy_(toks[(Wm + i) % n_sets])
             M.moe_layer(cfg, pool, dl.w_router, dl.bias, xbuf, out, ws, topk_idx_out=idx_log[i], opts=opts[i])
             ends[i].record(stream)
@@ -272,7 +288,7 @@ def gpu_arm(args, wl):
         barrier()
         torch.cuda.synchronize()
         for i in range(K):
-            flush.fill_(i & 0xFF)
+            flush_l2(i)
             e_s[i].record(stream)
             xbuf.copy_(hx[i % n_sets], non_blocking=True)
             M.moe_layer(cfg, pool, dl.w_router, dl.bias, xbuf, out, ws)
@@ -287,11 +303,19 @@ def gpu_arm(args, wl):
                "h2d_bytes_per_step": T * wl.d * toks.element_size(), "d2h_bytes_per_step": T * wl.d * 4,
                "api": "expert_ffn_router_b200.moe_layer (libmoe.so moe_layer), pinned host buffers"}
 
+    single = opts[0].n_launches == 1
+    router_bytes = wl.n_experts * wl.d * 4
     if rank == 0:
         hbm, which = peaks()
-        gu_avg_s = statistics.mean(gu_ms) / 1e3
-        gu_alg = statistics.mean(u * gu_bytes_e for u in uniq)
-        achieved = gu_alg / gu_avg_s / 1e9
+        if single:  # one kernel does the whole layer: its bytes are every expert's plus the router's
+            kname = "k_decode"
+            k_avg_s = statistics.mean(step_ms) / 1e3
+            k_alg = statistics.mean(u * (gu_bytes_e + dn_bytes_e) for u in uniq) + router_bytes
+        else:
+            kname = "k_gate_up"
+            k_avg_s = statistics.mean(gu_ms) / 1e3
+            k_alg = statistics.mean(u * gu_bytes_e for u in uniq)
+        achieved = k_alg / k_avg_s / 1e9
         traffic = None
         try:
             with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
@@ -301,8 +325,8 @@ def gpu_arm(args, wl):
                                                                                      "build.py"))
             B = importlib.util.module_from_spec(spec)
             spec.loader.exec_module(B)
-            if tr.get("source_hash") == B.source_hash() and tr.get("workload") == wl.name:
-                traffic = tr.get("k_gate_up_bytes_per_launch")
+            if tr.get("source_hash") == B.source_hash() and tr.get("workload") == wl.name and tr.get("kernel") == kname:
+                traffic = tr.get("bytes_per_launch")
         except Exception:
             traffic = None
         value = world * K * T / (max_ms / 1e3)
@@ -314,15 +338,16 @@ def gpu_arm(args, wl):
             "config": {"workload": wl.name, "T": T, "d": wl.d, "f": wl.f, "experts": wl.n_experts,
                        "shared": wl.has_shared, "top_k": wl.top_k, "wbits": wl.wbits,
                        "pool_gb": wl.pool_bytes / 1e9, "token_sets": n_sets,
-                       "l2": "flushed (256 MiB write) between timed steps, outside the per-step events",
+                       "l2": "flushed between timed steps (256 MiB write, then 256 MiB read), outside the per-step events",
                        "parallelism": f"replicas{world}"},
             "expert_weight_gbs": exp_gbs, "expert_weight_frac_of_8tbs": exp_gbs / NOMINAL_HBM_GBS,
             "expert_weight_frac_of_measured": exp_gbs / hbm, "unique_experts_per_step": statistics.mean(uniq),
-            "phase_ms": {"route": statistics.mean(route_ms), "gate_up": statistics.mean(gu_ms),
-                         "down_combine": statistics.mean(dn_ms)},
-            "roofline": {"kernel": "k_gate_up", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "phase_ms": ({"layer_single_launch": statistics.mean(step_ms)} if single else
+                         {"route": statistics.mean(route_ms), "gate_up": statistics.mean(gu_ms),
+                          "down_combine": statistics.mean(dn_ms)}),
+            "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "peak_source": which, "traffic": traffic,
-                         "alg_bytes_per_launch": gu_alg},
+                         "alg_bytes_per_launch": k_alg},
             "gpu_launches": launches,
             "clocks": clk.summary(),
         }
@@ -339,6 +364,8 @@ def main():
     args = parse()
     import workloads as W
     wl = W.workload(args.workload)
+    if args.n_experts:
+        wl = wl.replace(n_experts=args.n_experts, name=f"{wl.name}_e{args.n_experts}")
     if args.impl == "reference":
         reference_arm(args, wl)
     else:

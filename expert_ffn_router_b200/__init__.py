@@ -22,6 +22,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "moe.h")
 
 MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_ENOSPACE, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 MOE_F32, MOE_BF16 = 0, 1
+MOE_PATH_AUTO, MOE_PATH_MULTI, MOE_PATH_DECODE = 0, 1, 2
 
 
 class MoeError(RuntimeError):
@@ -49,7 +50,8 @@ class MoeConfig(ctypes.Structure):
 
 
 class MoeLayerOpts(ctypes.Structure):
-    _fields_ = [("events", ctypes.c_void_p * 4), ("n_launches", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+    _fields_ = [("events", ctypes.c_void_p * 4), ("path", ctypes.c_int32), ("n_launches", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 class MoePool(ctypes.Structure):

@@ -12,6 +12,7 @@
 
 #include "moe.h"
 #include "moe_launch.h"
+#include "moe_decode.cuh"
 #include "moe_route.cuh"
 
 namespace moe {
@@ -58,7 +59,9 @@ int persistent_grid(const void* func, size_t smem) {
 }
 
 cudaError_t allow_smem(const void* func, size_t smem) {
-    if (smem <= 48 * 1024) return cudaSuccess;
+    // dynamic + static shared memory above 48 KB needs the opt-in; static
+    // usage of these kernels is a few hundred bytes
+    if (smem + 4096 <= 48 * 1024) return cudaSuccess;
     int dev = 0;
     cudaGetDevice(&dev);
     const unsigned long long key = cache_key(dev, func, 0);
@@ -131,7 +134,9 @@ static Dims dims_of(const moe_config* c, int T, int S) {
 
 static int pick_ch(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8; }
 
-static Params base_params(const moe_config* c, const Dims& m, void* ws) {
+static Dims layout_dims(const moe_config* c, size_t ws_bytes);
+
+static Params base_params(const moe_config* c, const Dims& m, void* ws, size_t ws_bytes) {
     Params p{};
     p.m = m;
     p.routed_scale = c->routed_scale;
@@ -144,13 +149,21 @@ static Params base_params(const moe_config* c, const Dims& m, void* ws) {
     p.rb4 = kWarps * tl.rpw4;
     p.nrb4 = (c->d + p.rb4 - 1) / p.rb4;
     p.ksplit = 1;
-    p.ws = ws_carve(m, ws);
+    p.ws = ws_carve(layout_dims(c, ws_bytes), ws);
     return p;
 }
 
-static moe_status check_ws(const Dims& m, void* ws, size_t ws_bytes) {
+// The workspace layout: that of its capacity, independent of the call's T.
+static Dims layout_dims(const moe_config* c, size_t ws_bytes) {
+    Dims l = dims_of(c, 1, c->top_k + c->has_shared);
+    l.T = std::max(1, ws_capacity(l, ws_bytes));
+    return l;
+}
+
+static moe_status check_ws(const moe_config* c, int T, void* ws, size_t ws_bytes) {
     MOE_TRY(check_ptr(ws, "ws"));
-    const size_t need = ws_carve(m, nullptr).bytes;
+    Dims l = dims_of(c, std::max(1, T), c->top_k + c->has_shared);
+    const size_t need = ws_carve(l, nullptr).bytes;
     if (ws_bytes < need)
         return fail(MOE_ENOSPACE, "workspace has " + std::to_string(ws_bytes) + " bytes, needs " + std::to_string(need));
     return MOE_OK;
@@ -244,8 +257,10 @@ size_t moe_workspace_bytes(const moe_config* cfg, int32_t max_tokens) {
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
     MOE_TRY(check_ptr(ws, "ws"));
-    if (ws_bytes < sizeof(WsHeader)) return fail(MOE_ENOSPACE, "workspace smaller than its header");
-    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream);
+    if (ws_bytes < kCtrlBytes) return fail(MOE_ENOSPACE, "workspace smaller than its control words");
+    // every counter of the kernels (control words, per-task and per-row-block
+    // arrivals, running maxima) starts at zero and is left at zero by each call
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_workspace_init");
 }
 
@@ -282,8 +297,8 @@ moe_status moe_route(const moe_config* cfg, const void* x, moe_dtype dtype, int3
     MOE_TRY(check_ptr(topk_idx, "topk_idx"));
     MOE_TRY(check_ptr(topk_w, "topk_w"));
     const Dims m = dims_of(cfg, T, cfg->top_k + cfg->has_shared);
-    MOE_TRY(check_ws(m, ws, ws_bytes));
-    Params p = base_params(cfg, m, ws);
+    MOE_TRY(check_ws(cfg, T, ws, ws_bytes));
+    Params p = base_params(cfg, m, ws, ws_bytes);
     p.w_router = w_router;
     p.bias = bias;
     p.idx_out = topk_idx;
@@ -303,8 +318,8 @@ static moe_status expert_common(const moe_config* cfg, const moe_pool* pool, int
     if (expert == -1 && !cfg->has_shared) return fail(MOE_EINVAL, "no shared expert in this config");
     MOE_TRY(check_ptr(y, "y"));
     const Dims m = dims_of(cfg, T, 1);
-    MOE_TRY(check_ws(m, ws, ws_bytes));
-    Params p = base_params(cfg, m, ws);
+    MOE_TRY(check_ws(cfg, T, ws, ws_bytes));
+    Params p = base_params(cfg, m, ws, ws_bytes);
     p.pool = pool->w;
     p.scales = pool->s;
     p.direct_out = 1;
@@ -385,8 +400,8 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     MOE_TRY(check_ptr(topk_idx_out, "topk_idx_out", true));
     MOE_TRY(check_ptr(topk_w_out, "topk_w_out", true));
     const Dims m = dims_of(cfg, T, cfg->top_k + cfg->has_shared);
-    MOE_TRY(check_ws(m, ws, ws_bytes));
-    Params p = base_params(cfg, m, ws);
+    MOE_TRY(check_ws(cfg, T, ws, ws_bytes));
+    Params p = base_params(cfg, m, ws, ws_bytes);
     p.pool = pool->w;
     p.scales = pool->s;
     p.w_router = w_router;
@@ -401,7 +416,19 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         if (opts && opts->events[i]) return cudaEventRecord((cudaEvent_t)opts->events[i], s);
         return cudaSuccess;
     };
+    const int path = opts ? opts->path : MOE_PATH_AUTO;
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_MULTI && path != MOE_PATH_DECODE)
+        return fail(MOE_EINVAL, "opts->path must be MOE_PATH_AUTO, MOE_PATH_MULTI or MOE_PATH_DECODE");
+    DecPlan pl{};
+    const bool dec_ok = path != MOE_PATH_MULTI && decode_plan(m, &pl);
+    if (path == MOE_PATH_DECODE && !dec_ok) return fail(MOE_EINVAL, "shape does not fit the single-launch decode path");
     cudaError_t e = mark(0);
+    if (dec_ok) {
+        if (e == cudaSuccess) e = launch_decode(p, pl, x, dtype == MOE_BF16, s);
+        for (int i = 1; i < 4 && e == cudaSuccess; ++i) e = mark(i);
+        if (opts) opts->n_launches = 1;
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (decode)");
+    }
     if (e == cudaSuccess) e = launch_router_any(p, x, dtype, 1, 1, s);
     if (e == cudaSuccess) e = mark(1);
     if (e == cudaSuccess) e = launch_gate_up(p, tl, false, s);

@@ -16,8 +16,9 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // ---------------------------------------------------------------------------
 // Workspace: a 256-byte header of control words followed by the per-call
-// buffers.  Offsets depend on (cfg, T) only, so any workspace of at least
-// moe_workspace_bytes(cfg, T) bytes serves a call with T tokens.
+// buffers.  The layout is that of the workspace's capacity -- the largest
+// token count it can hold for the config (ws_capacity) -- so every call on one
+// workspace finds its counters at the same offsets whatever its own T.
 // ---------------------------------------------------------------------------
 struct WsHeader {
     int32_t status;       // first error code a kernel reported (0 = none)
@@ -27,12 +28,19 @@ struct WsHeader {
     int32_t n_asg;        // assignments incl. shared-expert ones
     int32_t n_items3;     // gate/up work items
     int32_t n_items4;     // down work items
-    int32_t pad[57];
+    uint32_t epoch;       // calls of the persistent decode kernel so far
+    uint32_t b1_count;    // its grid barrier: arrivals (self-resetting)
+    uint32_t b1_gen;      // its grid barrier: epoch of the last completion
+    int32_t pad[54];
 };
 static_assert(sizeof(WsHeader) == 256, "header must stay 256 bytes");
 
+constexpr int kReadyFlags = 2048;  // per-task ready flags of the decode kernel
+constexpr size_t kCtrlBytes = sizeof(WsHeader) + kReadyFlags * 4;  // zeroed by moe_workspace_init
+
 struct Ws {
     WsHeader* hdr;
+    uint32_t* ready;   // [kReadyFlags] epoch at which each task's hq became ready
     int8_t* xq;        // [T][d]     quantised activations
     float* sx;         // [T]        activation scales
     int32_t* xcs;      // [T]        sum of each token's codes
@@ -77,6 +85,7 @@ inline Ws ws_carve(const Dims& m, void* base) {
     };
     const size_t T = (size_t)m.T, A = (size_t)m.T * m.S;
     w.hdr = (WsHeader*)take(sizeof(WsHeader));
+    w.ready = (uint32_t*)take(kReadyFlags * 4);
     w.xq = (int8_t*)take(T * m.d);
     w.sx = (float*)take(T * 4);
     w.xcs = (int32_t*)take(T * 4);
@@ -94,6 +103,19 @@ inline Ws ws_carve(const Dims& m, void* base) {
     w.rb_ctr = (uint32_t*)take((size_t)((m.d + kMinRowBlock4 - 1) / kMinRowBlock4) * 4);
     w.bytes = off;
     return w;
+}
+
+// Largest T whose layout fits in `bytes` (0 if none): the layout of a
+// workspace is carved for this capacity, with S = top_k + has_shared slots.
+inline int ws_capacity(Dims m, size_t bytes) {
+    int lo = 0, hi = 1 << 20;
+    while (lo < hi) {
+        const int mid = lo + (hi - lo + 1) / 2;
+        m.T = mid;
+        if (ws_carve(m, nullptr).bytes <= bytes) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
 }
 
 // ---------------------------------------------------------------------------
@@ -160,6 +182,96 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 __device__ __forceinline__ void set_status(WsHeader* h, int code, int info) {
     if (atomicCAS(&h->status, 0, code) == 0) atomicExch(&h->status_info, info);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier / bulk-copy / ordering wrappers (sm_90+ PTX, used on sm_100a)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("{ .reg .b64 st; mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1; }" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// 1-D bulk copy global -> this CTA's shared memory, completion counted in bytes
+// on `bar`.  Addresses 16-byte aligned, size a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_volatile_status(const WsHeader* h) {
+    return *reinterpret_cast<const volatile int*>(&h->status);
+}
+
+// Bound of every device-side wait: after this long the waiter records
+// MOE_ETIMEOUT in the status word and stops waiting (as do all later waits of
+// the call, which see the status word set).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Wait for an mbarrier phase with a time bound; false if the wait gave up.
+// Unlike the flag waits this does not stop early when another wait has already
+// failed: the slots' bulk copies must still be waited for, so that no copy is
+// in flight into shared memory when the CTA exits.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            set_status(hdr, MOE_ETIMEOUT, site);
+            return false;
+        }
+    }
+    return true;
+}
+// Wait until *flag == want (acquire), with the same bound.
+__device__ __forceinline__ bool flag_wait_bounded(const uint32_t* flag, uint32_t want, WsHeader* hdr, int site) {
+    if (ld_acquire_u32(flag) == want) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_u32(flag) != want) {
+        if (ld_volatile_status(hdr) != 0) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            set_status(hdr, MOE_ETIMEOUT, site);
+            return false;
+        }
+        __nanosleep(64);
+    }
+    return true;
 }
 
 // ---------------------------------------------------------------------------

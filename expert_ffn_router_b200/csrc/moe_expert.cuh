@@ -158,6 +158,8 @@ __global__ void __launch_bounds__(kThreads) k_gate_up(const Params p) {
                     if (DBG && p.dbg_sh) p.dbg_sh[a] = sh;
                 }
             }
+            __syncthreads();  // every thread has read amax of the task's tokens
+            if (tid < n) p.ws.amax[s_asg[tid]] = 0u;  // leave the workspace zeroed for the next call
         }
     }
     (void)redi;

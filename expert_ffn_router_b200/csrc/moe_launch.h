@@ -20,6 +20,12 @@ int persistent_grid(const void* func, size_t smem);
 // Raise the dynamic shared-memory limit of a kernel once (cached).
 cudaError_t allow_smem(const void* func, size_t smem);
 
+struct DecPlan;
+// Persistent single-launch decode kernel (T <= 8): plan (false if the shape
+// does not fit) and cooperative launch.
+bool decode_plan(const Dims& m, DecPlan* pl);
+cudaError_t launch_decode(const Params& p, const DecPlan& pl, const void* x, bool bf16, cudaStream_t s);
+
 cudaError_t launch_gate_up(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s);
 cudaError_t launch_down(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s);
 

@@ -98,9 +98,9 @@ typedef struct {
 /* Bytes of workspace the calls below need for up to max_tokens tokens. */
 MOE_API size_t moe_workspace_bytes(const moe_config* cfg, int32_t max_tokens);
 
-/* Zero the workspace control words.  Call once after allocating a workspace
- * (and after a call that reported a device error) before its first use; the
- * kernels leave the control words at zero between calls. */
+/* Zero the whole workspace (its control words and counters).  Call once after
+ * allocating a workspace, and again after a call that reported a device error,
+ * before its next use; the kernels leave every counter at zero between calls. */
 MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Activation quantiser alone (step a0), exposed for parity checks.
@@ -146,11 +146,18 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *  events: cudaEvent_t handles (or NULL) recorded on `stream` before routing
  *          [0], after routing and bucketing [1], after gate/up [2] and after
  *          down + combine [3]; for timing the phases on the launching stream.
+ *          The single-launch decode path records [0] before and [1..3] after
+ *          its one kernel.
+ *  path: MOE_PATH_AUTO (0), MOE_PATH_MULTI (1: separate routing, gate/up and
+ *        down kernels) or MOE_PATH_DECODE (2: one persistent kernel for
+ *        T <= 8; MOE_EINVAL if the shape does not fit it).
  *  n_launches: set to the number of kernels the call launched. */
+enum { MOE_PATH_AUTO = 0, MOE_PATH_MULTI = 1, MOE_PATH_DECODE = 2 };
 typedef struct {
     void* events[4];
+    int32_t path;
     int32_t n_launches;
-    int32_t reserved[7];
+    int32_t reserved[6];
 } moe_layer_opts;
 
 /* moe_layer with options (opts may be NULL, then identical to moe_layer). */

@@ -25,7 +25,13 @@ SMALL = {
     "k_eq_E": W.workload(0).replace(name="k_eq_E", d=256, f=128, n_experts=4, top_k=4, T=9),
     "no_shared": W.workload(0).replace(name="no_shared", d=512, f=256, n_experts=16, top_k=3, T=3,
                                        has_shared=0),
+    "tiny_T1": W.workload(0).replace(name="tiny", T=1),
+    "tiny_T8": W.workload(0).replace(name="tiny", T=8),
+    "ragged_int2_T2": W.workload(0).replace(name="ragged_int2", d=1088, f=320, n_experts=24, top_k=5, T=2,
+                                            wbits=2),
+    "wide_k": W.workload(0).replace(name="wide_k", d=256, f=96, n_experts=64, top_k=32, T=7),
 }
+PATHS = {"auto": M.MOE_PATH_AUTO, "multi": M.MOE_PATH_MULTI}
 
 
 def cfg_of(wl):
@@ -48,7 +54,7 @@ def assert_ok(ws):
 def test_quantize_bitexact(name):
     wl = SMALL.get(name) or W.workload(1)
     x = x_host(wl, 3, 64 if name == "bf16_d6144" else None)
-    x[1].zero_()  # an all-zero token
+    x[x.shape[0] // 2].zero_()  # an all-zero token
     q_o, s_o = O.quantize(x.float())
     xq = torch.empty(x.shape, dtype=torch.int8, device="cuda")
     sx = torch.empty(x.shape[0], dtype=torch.float32, device="cuda")
@@ -139,17 +145,21 @@ def test_expert_stages(name, T, expert):
     assert rel_l2(y.cpu().numpy(), r["y"]) <= OUT_REL_L2
 
 
-def run_layer_gpu(wl, dl, x, accumulate_into=None):
+def run_layer_gpu(wl, dl, x, accumulate_into=None, path="auto", ws=None):
     cfg = cfg_of(wl)
     T = x.shape[0]
     pool = M.make_pool(dl.pool_w, dl.pool_s)
     out = accumulate_into if accumulate_into is not None else torch.empty(T, wl.d, device="cuda")
     idx = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
     w = torch.empty(T, wl.top_k, device="cuda")
-    ws = M.workspace(cfg, T)
+    ws = M.workspace(cfg, T) if ws is None else ws
+    opts = M.MoeLayerOpts()
+    opts.path = PATHS[path]
     M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x), out, ws, accumulate=accumulate_into is not None,
-                topk_idx_out=idx, topk_w_out=w)
+                topk_idx_out=idx, topk_w_out=w, opts=opts)
     assert_ok(ws)
+    if path == "auto" and T <= 8:
+        assert opts.n_launches == 1  # the single-launch decode kernel ran
     return out, idx.cpu().numpy(), w.cpu().numpy()
 
 
@@ -169,32 +179,50 @@ def compare_layer(wl, L, x, out, g_idx, tokens=None):
     return err, allowed
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", list(SMALL))
-def test_layer_small(name):
+def test_layer_small(name, path):
     wl = SMALL[name]
     L = W.layer(wl, 0, 0)
     dl = W.device_layer(wl, 0, 0, host=L)
     x = x_host(wl)
-    out, g_idx, _ = run_layer_gpu(wl, dl, x)
+    out, g_idx, _ = run_layer_gpu(wl, dl, x, path=path)
     compare_layer(wl, L, x, out, g_idx)
     # accumulate mode adds the layer to what is there
     base = torch.randn(x.shape[0], wl.d, device="cuda")
-    acc, _, _ = run_layer_gpu(wl, dl, x, accumulate_into=base.clone())
+    acc, _, _ = run_layer_gpu(wl, dl, x, accumulate_into=base.clone(), path=path)
     np.testing.assert_allclose(acc.cpu().numpy(), (base + out).cpu().numpy(), rtol=1e-6, atol=1e-5)
 
 
 def test_layer_decode_full_size():
-    """The decode workload as the bench runs it: T = 1 per call, 8 token sets."""
+    """The decode workload as the bench runs it: T = 1 per call, 8 token sets,
+    one workspace reused across calls; then T = 8, and the multi-kernel path."""
     wl = W.workload(1)
     L = W.layer(wl, 0, 0)
     dl = W.device_layer(wl, 0, 0, host=L)
+    ws = M.workspace(cfg_of(wl), 8)
     errs = []
     for s in range(8):
         x = x_host(wl, s)
-        out, g_idx, _ = run_layer_gpu(wl, dl, x)
+        out, g_idx, _ = run_layer_gpu(wl, dl, x, ws=ws)
         err, allowed = compare_layer(wl, L, x, out, g_idx)
         errs.append(err)
-    print("decode rel L2 per token:", errs)
+    x = x_host(wl, 20, 8)
+    out, g_idx, _ = run_layer_gpu(wl, dl, x, ws=ws)
+    errs.append(compare_layer(wl, L, x, out, g_idx)[0])
+    out, g_idx, _ = run_layer_gpu(wl, dl, x_host(wl, 0), path="multi", ws=ws)
+    errs.append(compare_layer(wl, L, x_host(wl, 0), out, g_idx)[0])
+    print("decode rel L2 per call:", errs)
+
+
+def test_layer_decode_int2_full_size():
+    wl = W.workload(4)
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    for T in (1, 3):
+        x = x_host(wl, 5, T)
+        out, g_idx, _ = run_layer_gpu(wl, dl, x)
+        compare_layer(wl, L, x, out, g_idx)
 
 
 def test_layer_prefill_sampled():
@@ -255,7 +283,7 @@ def test_workspace_reuse_and_status():
     ws = M.workspace(cfg, wl.T)
     pool = M.make_pool(dl.pool_w, dl.pool_s)
     outs = []
-    for T in (wl.T, 1, 5, wl.T):
+    for T in (wl.T, 1, 5, wl.T, 5):  # alternates the multi-kernel and the single-launch paths
         x = to_dev(x_host(wl, T, T))
         out = torch.empty(T, wl.d, device="cuda")
         M.moe_layer(cfg, pool, dl.w_router, dl.bias, x, out, ws)
@@ -266,3 +294,4 @@ def test_workspace_reuse_and_status():
     M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x_host(wl, wl.T, wl.T)), ref, ws2)
     torch.cuda.synchronize()
     assert torch.equal(outs[0], ref) and torch.equal(outs[3], ref)  # deterministic
+    assert torch.equal(outs[2], outs[4])
