@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--trace", default="", help="write per-CTA phase stamps of one extra step to this JSON file")
     ap.add_argument("--n-experts", type=int, default=0,
                     help="profiling case: the same layer with fewer routed experts (smaller pool)")
     return ap.parse_args()
@@ -181,6 +182,38 @@ def reference_arm(args, wl):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+TRACE_NAMES = {0: "start", 1: "quantised", 2: "router_done", 3: "shared_gate_up_done", 4: "grid_barrier",
+               5: "routing_done", 6: "routed_gate_up_done", 7: "first_down_staged", 8: "down_done",
+               9: "cons_wait_full_total", 10: "prod_wait_empty_total",
+               12: "prod_pre_routing_issued", 13: "prod_routing_received", 14: "prod_all_issued",
+               15: "prod_drained"}
+
+
+def write_trace(path, M, cfg, pool, dl, xbuf, out, ws, dev, flush_l2):
+    """One extra step of the single-launch path with the phase trace on; writes
+    per-phase stamps (us after the earliest CTA start) as min/median/max over CTAs."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tr = torch.zeros(sms, 16, dtype=torch.int64, device=dev)
+    o = M.MoeLayerOpts()
+    o.trace = tr.data_ptr()
+    flush_l2(0)
+    M.moe_layer(cfg, pool, dl.w_router, dl.bias, xbuf, out, ws, opts=o)
+    torch.cuda.synchronize()
+    t = tr.cpu().numpy().astype("float64")
+    t0 = t[:, 0].min()
+    rec = {}
+    for i, name in TRACE_NAMES.items():
+        col = t[:, i]
+        col = col[col > 0]
+        if col.size:
+            v = (col - (0 if name.endswith("_total") else t0)) / 1e3
+            rec[name] = {"min": float(v.min()), "median": float(sorted(v)[len(v) // 2]), "max": float(v.max())}
+    raw = ((t - t0) / 1e3).round(3).tolist()
+    with open(path, "w") as fh:
+        json.dump({"us_after_first_cta_start": rec, "ctas": int(sms), "raw_us": raw}, fh)
+
+
 def gpu_arm(args, wl):
     import numpy as np
     import torch
@@ -305,6 +338,8 @@ def gpu_arm(args, wl):
 
     single = opts[0].n_launches == 1
     router_bytes = wl.n_experts * wl.d * 4
+    if args.trace and rank == 0:
+        write_trace(args.trace, M, cfg, pool, dl, xbuf, out, ws, dev, flush_l2)
     if rank == 0:
         hbm, which = peaks()
         if single:  # one kernel does the whole layer: its bytes are every expert's plus the router's

@@ -51,7 +51,7 @@ class MoeConfig(ctypes.Structure):
 
 class MoeLayerOpts(ctypes.Structure):
     _fields_ = [("events", ctypes.c_void_p * 4), ("path", ctypes.c_int32), ("n_launches", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("trace", ctypes.c_void_p), ("reserved", ctypes.c_int32 * 4)]
 
 
 class MoePool(ctypes.Structure):

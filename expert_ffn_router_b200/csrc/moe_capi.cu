@@ -149,7 +149,9 @@ static Params base_params(const moe_config* c, const Dims& m, void* ws, size_t w
     p.rb4 = kWarps * tl.rpw4;
     p.nrb4 = (c->d + p.rb4 - 1) / p.rb4;
     p.ksplit = 1;
-    p.ws = ws_carve(layout_dims(c, ws_bytes), ws);
+    const Dims l = layout_dims(c, ws_bytes);
+    p.ws = ws_carve(l, ws);
+    p.a_cap = l.T * l.S;
     return p;
 }
 
@@ -410,6 +412,7 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     p.accumulate = accumulate ? 1 : 0;
     p.idx_out = topk_idx_out;
     p.w_out = topk_w_out;
+    p.trace = opts ? static_cast<unsigned long long*>(opts->trace) : nullptr;
     cudaStream_t s = (cudaStream_t)stream;
     const ExpertTiling tl = expert_tiling(cfg->d, cfg->f, cfg->wbits);
     auto mark = [&](int i) -> cudaError_t {

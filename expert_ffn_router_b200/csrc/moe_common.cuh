@@ -51,6 +51,7 @@ struct Ws {
     int4* tasks;       // [max_tasks] (blob, asg start, n tokens, 0)
     uint32_t* task_ctr;// [max_tasks] gate/up item arrivals per task (self-resetting)
     uint32_t* amax;    // [T*S]      max |h| per assignment (float bits)
+    uint32_t* amax2;   // [T*S]      second copy: the decode kernel alternates by call parity
     float* h;          // [T*S][f]   SwiGLU output
     int8_t* hq;        // [T*S][f]   requantised h
     float* sh;         // [T*S]      scale of hq
@@ -96,6 +97,7 @@ inline Ws ws_carve(const Dims& m, void* base) {
     w.tasks = (int4*)take((size_t)max_tasks(m) * 16);
     w.task_ctr = (uint32_t*)take((size_t)max_tasks(m) * 4);
     w.amax = (uint32_t*)take(A * 4);
+    w.amax2 = (uint32_t*)take(A * 4);
     w.h = (float*)take(A * m.f * 4);
     w.hq = (int8_t*)take(A * m.f);
     w.sh = (float*)take(A * 4);
@@ -133,6 +135,8 @@ struct Params {
     int rb4, nrb4;   // down rows per item, items per task
     int ksplit;      // router split of d
     Ws ws;
+    int a_cap;       // assignments the workspace layout holds (capacity T x S)
+    unsigned long long* trace;  // optional per-CTA phase stamps of the decode kernel
     const float* w_router;
     const float* bias;
     float* out;

@@ -1,13 +1,14 @@
 // The whole MoE layer for decode-sized batches (T <= 8) in one persistent,
-// cooperatively launched kernel: one CTA per SM, 8 consumer warps and one
-// producer warp.
+// cooperatively launched kernel: one CTA per SM, two groups of 8 consumer
+// warps and one producer warp.
 //
 // The producer streams every weight row the CTA needs -- its router rows, its
 // share of the shared expert's gate/up rows, then (once the routing is known)
 // its share of the routed gate/up rows and of all down rows -- into a ring of
 // shared-memory slots with 1-D bulk copies (cp.async.bulk, completion counted
 // on an mbarrier per slot).  The consumers work through the same unit
-// sequence:
+// sequence, the two consumer groups taking alternate units (4 warps per
+// scheduler to hide the dot products' latencies):
 //   1. quantise the T tokens (every CTA, into its own shared memory);
 //   2. router units: logits of this CTA's experts -> workspace; arrive at the
 //      one grid barrier;
@@ -16,8 +17,9 @@
 //      top-k routing and the same expert task list (no second barrier);
 //   5. routed gate/up units; the warp that completes a task's last row
 //      requantises its h and publishes the task as ready (release flag);
-//   6. down units (waiting, bounded, for their task's ready flag); the warp
-//      that completes a row block's last contribution combines it.
+//   6. down units (waiting, bounded, for their task's ready flag); at the end
+//      each CTA signs its row blocks off and the CTA bringing a row block's
+//      last task combines it.
 // Each expert selected by several tokens is streamed once: a task is one
 // expert with all its tokens.  Every wait is bounded (MOE_ETIMEOUT).
 #pragma once
@@ -28,21 +30,27 @@
 
 namespace moe {
 
-constexpr int kDecWarps = 8;
-constexpr int kDecThreads = (kDecWarps + 1) * 32;
-constexpr int kDecCons = kDecWarps * 32;
-constexpr int kDecMaxSlots = 4;
+constexpr int kDecWarps = 8;                         // warps of a consumer group = rows per gate/up unit
+constexpr int kDecGroups = 2;
+constexpr int kDecConsWarps = kDecWarps * kDecGroups;
+constexpr int kDecThreads = (kDecConsWarps + 1) * 32;
+constexpr int kDecCons = kDecConsWarps * 32;           // consumer threads
+constexpr int kDecGrp = kDecWarps * 32;                // threads of one group
+constexpr int kDecMaxSlots = 4;  // ring slots; always even (see decode_plan)
 constexpr int kDecMaxT = 8;
 constexpr int kDecMaxK = 32;
 constexpr int kDecMaxTasks = kDecMaxT * kDecMaxK + 1;
-constexpr int kDecBar = 1;  // named barrier of the consumer warps
+constexpr int kDecBiasCache = 256;  // experts whose bias the kernel keeps in shared memory
+constexpr int kDecBar = 1;  // named barrier of all consumer warps; 2 + g: group g
 
 struct DecPlan {
     int slot_bytes, nslot;
+    int wbytes;        // weight bytes of a slot; the row scales follow at this offset
     int rd;            // down rows per unit (multiple of kDecWarps)
     int rr;            // router rows per unit (1 or 2)
     int nu_gu, nu_dn;  // units per task
     int xs_off, hs_off, ring_off, smem_bytes;
+    int hs_grp_bytes;  // h staging bytes of one consumer group (T * f)
 };
 
 struct DecCtl {
@@ -51,22 +59,26 @@ struct DecCtl {
     uint64_t route_ready;
     uint32_t epoch;
     int n_tasks;
-    int hq_task;
+    int hq_task[kDecGroups];
+    int n_last;
     float sx[kDecMaxT];
     int xcs[kDecMaxT];
     int idx[kDecMaxT][kDecMaxK];
     float w[kDecMaxT][kDecMaxK];
     int4 tasks[kDecMaxTasks];  // (blob, n tokens, -, -)
     int ttok[kDecMaxTasks][kDecMaxT];
-    int sorted[kDecMaxT * kDecMaxK];
-    int hcs[kDecMaxT];
-    float hsh[kDecMaxT];
-    float redf[kDecWarps];
-    int redi[kDecWarps];
-    float part[kDecWarps][2 * kDecMaxT];
+    int sorted[kDecMaxT * kDecMaxK];    // assignment ids by (expert, token, slot)
+    int sorted_e[kDecMaxT * kDecMaxK];  // their experts
+    int hcs[kDecGroups][kDecMaxT];
+    float hsh[kDecGroups][kDecMaxT];
+    int last_rb[kDecCons];
+    float bias_s[kDecBiasCache];  // the router bias (E <= kDecBiasCache)
+    float redf[kDecConsWarps];
+    int redi[kDecConsWarps];
+    float part[kDecGroups][kDecWarps][2 * kDecMaxT];
 };
 
-// --- consumer-only reductions (named barrier, 256 threads) -----------------
+// --- consumer reductions over all consumer warps (named barrier 1) ---------
 __device__ __forceinline__ float cons_max(float v, float* red) {
     v = warp_max(v);
     named_sync(kDecBar, kDecCons);
@@ -74,7 +86,7 @@ __device__ __forceinline__ float cons_max(float v, float* red) {
     named_sync(kDecBar, kDecCons);
     float r = red[0];
 #pragma unroll
-    for (int i = 1; i < kDecWarps; ++i) r = fmaxf(r, red[i]);
+    for (int i = 1; i < kDecConsWarps; ++i) r = fmaxf(r, red[i]);
     return r;
 }
 __device__ __forceinline__ int cons_sum_int(int v, int* red) {
@@ -84,8 +96,47 @@ __device__ __forceinline__ int cons_sum_int(int v, int* red) {
     named_sync(kDecBar, kDecCons);
     int r = 0;
 #pragma unroll
-    for (int i = 0; i < kDecWarps; ++i) r += red[i];
+    for (int i = 0; i < kDecConsWarps; ++i) r += red[i];
     return r;
+}
+// ... and over one group's 8 warps (named barrier 2 + g); red has kDecConsWarps entries
+__device__ __forceinline__ int grp_sum_int(int v, int* red, int g) {
+    v = __reduce_add_sync(kFull, v);
+    named_sync(2 + g, kDecGrp);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    named_sync(2 + g, kDecGrp);
+    int r = 0;
+#pragma unroll
+    for (int i = 0; i < kDecWarps; ++i) r += red[g * kDecWarps + i];
+    return r;
+}
+
+// One 16-byte weight chunk against one activation chunk held in registers
+// (x[s] = sub-array s of the staged layout), into two accumulators (even and
+// odd weight words) to halve the dependent dp4a chain.
+template <int WB>
+__device__ __forceinline__ void dot_chunk_regs(const uint4 w, const uint4* x, int& a0, int& a1) {
+    if (WB == 4) {
+        const unsigned p = w.x ^ 0x88888888u, q = w.y ^ 0x88888888u;
+        const unsigned r = w.z ^ 0x88888888u, t = w.w ^ 0x88888888u;
+        a0 = dp4a_us(p & 0x0F0F0F0Fu, (int)x[0].x, a0);
+        a1 = dp4a_us((p >> 4) & 0x0F0F0F0Fu, (int)x[0].y, a1);
+        a0 = dp4a_us(q & 0x0F0F0F0Fu, (int)x[0].z, a0);
+        a1 = dp4a_us((q >> 4) & 0x0F0F0F0Fu, (int)x[0].w, a1);
+        a0 = dp4a_us(r & 0x0F0F0F0Fu, (int)x[1].x, a0);
+        a1 = dp4a_us((r >> 4) & 0x0F0F0F0Fu, (int)x[1].y, a1);
+        a0 = dp4a_us(t & 0x0F0F0F0Fu, (int)x[1].z, a0);
+        a1 = dp4a_us((t >> 4) & 0x0F0F0F0Fu, (int)x[1].w, a1);
+    } else {
+        const unsigned ws[4] = {w.x ^ 0xAAAAAAAAu, w.y ^ 0xAAAAAAAAu, w.z ^ 0xAAAAAAAAu, w.w ^ 0xAAAAAAAAu};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            a0 = dp4a_us(ws[s] & 0x03030303u, (int)x[s].x, a0);
+            a1 = dp4a_us((ws[s] >> 2) & 0x03030303u, (int)x[s].y, a1);
+            a0 = dp4a_us((ws[s] >> 4) & 0x03030303u, (int)x[s].z, a0);
+            a1 = dp4a_us((ws[s] >> 6) & 0x03030303u, (int)x[s].w, a1);
+        }
+    }
 }
 
 // 16 consecutive activations (i a multiple of 16) as floats.
@@ -147,7 +198,68 @@ __device__ __forceinline__ void topk_warp(const float* lrow, const float* bias, 
     my_w = lane < k ? __fmul_rn(__fdiv_rn(my_s, ssum), scale) : 0.0f;
 }
 
-template <int WB, int TM, typename XT>
+// NG / ND: 16-byte weight chunks per lane of a gate/up row / a down row when
+// the row is exactly 32 * NG (32 * ND) chunks (fully unrolled, weights loaded
+// up front); 0 = any shape (runtime loop).
+// Order-preserving map of a float to an unsigned key (larger float, larger key).
+__device__ __forceinline__ unsigned float_key(float v) {
+    const unsigned b = __float_as_uint(v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Top-k of one token by one warp for E <= 256: lane l holds experts l + 32 i
+// in registers; each round takes the largest selection score (lowest index on
+// ties) with two warp reductions.  Same rule and arithmetic as topk_warp.
+__device__ __forceinline__ void topk_warp_small(const float* lrow, const float* bias_s, int E, int k, float scale,
+                                                int& my_e, float& my_w) {
+    const int lane = threadIdx.x & 31;
+    float sv[8];
+    unsigned key[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        sv[i] = 0.0f;
+        key[i] = 0u;  // below every real key
+        if (e < E) {
+            const float lg = __ldcg(lrow + e);
+            sv[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-lg)));
+            key[i] = float_key(__fadd_rn(sv[i], bias_s[e]));
+        }
+    }
+    float ssum = 0.0f, my_s = 0.0f;
+    my_e = 0;
+    for (int j = 0; j < k; ++j) {
+        unsigned best = 0u;
+        int bi = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (key[i] > best) {  // ascending index within the lane: strict keeps the lower one
+                best = key[i];
+                bi = i;
+            }
+        const unsigned mx = __reduce_max_sync(kFull, best);
+        const int e_win = __reduce_min_sync(kFull, best == mx ? lane + 32 * bi : 0x7fffffff);
+        const int owner = e_win & 31, slot = e_win >> 5;
+        float s_mine = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i == slot) s_mine = sv[i];
+        const float sj = __shfl_sync(kFull, s_mine, owner);
+        if (lane == owner) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i == slot) key[i] = 0u;
+        }
+        if (lane == j) {
+            my_e = e_win;
+            my_s = sj;
+        }
+        ssum = __fadd_rn(ssum, sj);
+    }
+    my_w = lane < k ? __fmul_rn(__fdiv_rn(my_s, ssum), scale) : 0.0f;
+}
+
+template <int WB, int TM, int NG, int ND, typename XT>
 __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const DecPlan pl, const XT* __restrict__ x) {
     constexpr int NSUB = 8 / WB;
     extern __shared__ __align__(128) uint8_t dec_smem[];
@@ -162,6 +274,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     const int nch_gu = rb_gu / 16, nch_dn = rb_dn / 16;
     const int nslot = pl.nslot, slot_bytes = pl.slot_bytes;
     WsHeader* hdr = p.ws.hdr;
+    unsigned long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * 16 : nullptr;
+#define DEC_TRACE(i)                                   \
+    do {                                               \
+        if (trace) trace[i] = global_timer_ns();       \
+    } while (0)
 
     if (tid == 0) {
         for (int i = 0; i < nslot; ++i) {
@@ -171,86 +288,141 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         mbar_init(&C.route_ready, 1);
         fence_mbar_init();
         C.epoch = __ldcg(&hdr->epoch);
-        C.hq_task = -1;
+        for (int g = 0; g < kDecGroups; ++g) C.hq_task[g] = -1;
     }
     __syncthreads();  // the only CTA-wide barrier: producer and consumers part here
     const uint32_t epoch = C.epoch;
+    // running maxima of |h| alternate between two arrays by call parity; each
+    // call zeroes the one the next call uses
+    uint32_t* amax_cur = (epoch & 1) ? p.ws.amax2 : p.ws.amax;
+    uint32_t* amax_nxt = (epoch & 1) ? p.ws.amax : p.ws.amax2;
+    if (tid == 0) DEC_TRACE(0);
     const int n_my_router = c < E ? (E - c + G - 1) / G : 0;  // experts c, c+G, ...
     const int n_router_units = (n_my_router + pl.rr - 1) / pl.rr;
     const int n_sh_units = HS && c < pl.nu_gu ? (pl.nu_gu - c + G - 1) / G : 0;  // shared units c, c+G, ...
 
     // =====================================================================
-    // producer: lane 0 of warp kDecWarps
+    // producer: lane 0 of the last warp
     // =====================================================================
-    if (warp == kDecWarps) {
+    if (warp == kDecConsWarps) {
         if (lane != 0) return;
-        uint32_t u = 0;
+        // ring position of the next unit, advanced without divisions
+        int ps = 0;          // slot
+        uint32_t pr = 0;     // round of that slot (times it has been filled before)
+        uint32_t issued = 0; // units issued
+        unsigned long long t_empty = 0;  // time blocked on free slots (traced)
         auto take = [&](uint32_t bytes) -> uint8_t* {
-            const int s = u % nslot;
-            const uint32_t round = u / nslot;
-            if (round > 0) mbar_wait_bounded(&C.empty[s], (round - 1) & 1, hdr, 100 + s);
-            mbar_arrive_expect_tx(&C.full[s], bytes);
-            return ring + (size_t)s * slot_bytes;
+            if (pr > 0) {
+                const unsigned long long t0 = trace ? global_timer_ns() : 0;
+                mbar_wait_bounded(&C.empty[ps], (pr - 1) & 1, hdr, 100 + ps);
+                if (trace) t_empty += global_timer_ns() - t0;
+            }
+            mbar_arrive_expect_tx(&C.full[ps], bytes);
+            return ring + (size_t)ps * slot_bytes;
+        };
+        auto advance = [&]() {
+            ++issued;
+            if (++ps == nslot) {
+                ps = 0;
+                ++pr;
+            }
         };
         const int n_blobs = E + HS;
         auto issue_gu = [&](int blob, int j) {
             blob = min(max(blob, 0), n_blobs - 1);  // never copy outside the pool, whatever happened
-            const int r0 = j * kDecWarps, rows = min(kDecWarps, f - r0);
+            const int r0 = j * kDecWarps, rows = min(kDecWarps, f - r0);  // f % 8 == 0: rows == 8
             const uint32_t bytes = (uint32_t)rows * rb_gu;
             const uint8_t* base = p.pool + (size_t)blob * p.blob_bytes;
-            uint8_t* dst = take(2 * bytes);
-            bulk_g2s(dst, base + (size_t)r0 * rb_gu, bytes, &C.full[u % nslot]);
-            bulk_g2s(dst + (size_t)kDecWarps * rb_gu, base + ((size_t)f + r0) * rb_gu, bytes, &C.full[u % nslot]);
-            ++u;
+            const float* sc = p.scales + (size_t)blob * p.scale_rows;
+            uint64_t* bar = &C.full[ps];
+            uint8_t* dst = take(2 * bytes + 2 * rows * 4);
+            bulk_g2s(dst, base + (size_t)r0 * rb_gu, bytes, bar);
+            bulk_g2s(dst + (size_t)kDecWarps * rb_gu, base + ((size_t)f + r0) * rb_gu, bytes, bar);
+            bulk_g2s(dst + pl.wbytes, sc + r0, rows * 4, bar);                      // gate row scales
+            bulk_g2s(dst + pl.wbytes + kDecWarps * 4, sc + f + r0, rows * 4, bar);  // up row scales
+            advance();
         };
         for (int ru = 0; ru < n_router_units; ++ru) {
             const int rows = min(pl.rr, n_my_router - ru * pl.rr);
             uint8_t* dst = take((uint32_t)rows * d * 4);
             for (int i = 0; i < rows; ++i) {
                 const int e = c + (ru * pl.rr + i) * G;
-                bulk_g2s(dst + (size_t)i * d * 4, p.w_router + (size_t)e * d, (uint32_t)d * 4, &C.full[u % nslot]);
+                bulk_g2s(dst + (size_t)i * d * 4, p.w_router + (size_t)e * d, (uint32_t)d * 4, &C.full[ps]);
             }
-            ++u;
+            advance();
         }
         for (int i = 0; i < n_sh_units; ++i) issue_gu(E, c + i * G);
+        DEC_TRACE(12);
         mbar_wait_bounded(&C.route_ready, 0, hdr, 110);
+        DEC_TRACE(13);
         const int n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
-        const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
-        for (long long g = c * Nr / G; g < (c + 1) * Nr / G; ++g)
-            issue_gu(C.tasks[HS + (int)(g / pl.nu_gu)].x, (int)(g % pl.nu_gu));
-        const long long Nd = (long long)n_tasks * pl.nu_dn;
-        for (long long g = c * Nd / G; g < (c + 1) * Nd / G; ++g) {
-            const int blob = min(max(C.tasks[(int)(g / pl.nu_dn)].x, 0), n_blobs - 1), j = (int)(g % pl.nu_dn);
-            const int r0 = j * pl.rd, rows = min(pl.rd, d - r0);
-            const uint32_t bytes = (uint32_t)rows * rb_dn;
-            uint8_t* dst = take(bytes);
-            bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)r0 * rb_dn, bytes,
-                     &C.full[u % nslot]);
-            ++u;
+        {
+            const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
+            const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
+            int ti = HS + (int)(lo / pl.nu_gu), j = (int)(lo % pl.nu_gu);
+            for (long long g = lo; g < hi; ++g) {
+                issue_gu(C.tasks[ti].x, j);
+                if (++j == pl.nu_gu) {
+                    j = 0;
+                    ++ti;
+                }
+            }
         }
+        {
+            const long long Nd = (long long)n_tasks * pl.nu_dn;
+            const long long lo = c * Nd / G, hi = (c + 1) * Nd / G;
+            int ti = (int)(lo / pl.nu_dn), j = (int)(lo % pl.nu_dn);
+            for (long long g = lo; g < hi; ++g) {
+                const int blob = min(max(C.tasks[ti].x, 0), n_blobs - 1);
+                const int r0 = j * pl.rd, rows = min(pl.rd, d - r0);  // multiples of 8
+                const uint32_t bytes = (uint32_t)rows * rb_dn;
+                uint64_t* bar = &C.full[ps];
+                uint8_t* dst = take(bytes + rows * 4);
+                bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)r0 * rb_dn, bytes,
+                         bar);
+                bulk_g2s(dst + pl.wbytes, p.scales + (size_t)blob * p.scale_rows + 2 * f + r0, rows * 4, bar);
+                advance();
+                if (++j == pl.nu_dn) {
+                    j = 0;
+                    ++ti;
+                }
+            }
+        }
+        DEC_TRACE(14);
+        if (trace) trace[10] = t_empty;
         // drain: every copy issued must have landed before this thread (and so
         // the CTA and its shared memory) can retire
         for (int s = 0; s < nslot; ++s)
-            if (u > (uint32_t)s) mbar_wait_bounded(&C.full[s], ((u - s + nslot - 1) / nslot - 1) & 1, hdr, 120 + s);
+            if (issued > (uint32_t)s)
+                mbar_wait_bounded(&C.full[s], ((issued - s + nslot - 1) / nslot - 1) & 1, hdr, 120 + s);
+        DEC_TRACE(15);
         return;
     }
 
     // =====================================================================
-    // consumers: warps 0..7, ctid = threadIdx.x
+    // consumers: warps 0..15, two groups of 8; unit u belongs to group u & 1
     // =====================================================================
     const int ctid = tid;
+    const int grp = warp / kDecWarps, gw = warp % kDecWarps, gtid = ctid % kDecGrp;
+    const int hs_grp = pl.hs_grp_bytes;  // staging bytes of one group
+
     // ---- 1. quantise the T tokens into the permuted staging layout ----
+    if (E <= kDecBiasCache)
+        for (int e = ctid; e < E; e += kDecCons) C.bias_s[e] = __ldg(p.bias + e);
     for (int t = 0; t < T; ++t) {
         const XT* xt = x + (size_t)t * d;
+        float v[16];
         float m = 0.0f;
-        for (int col = ctid; col < d; col += kDecCons) m = fmaxf(m, fabsf(load_x(xt, col)));
+        const int pc = ctid;  // d / 16 <= kDecCons pieces of 16 values
+        if (pc < d / 16) {
+            load16(xt, (size_t)pc * 16, v);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) m = fmaxf(m, fabsf(v[q]));
+        }
         m = cons_max(m, C.redf);
         const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
         int cs = 0;
-        uint4* xst = xs + (size_t)t * NSUB * nch_gu;
-        for (int pc = ctid; pc < d / 16; pc += kDecCons) {
-            float v[16];
-            load16(xt, (size_t)pc * 16, v);
+        if (pc < d / 16) {
             unsigned wds[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
@@ -258,7 +430,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 cs += code;
                 wds[q >> 2] |= ((unsigned)code & 0xFFu) << (8 * (q & 3));
             }
-            xst[(pc % NSUB) * nch_gu + pc / NSUB] = permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
+            xs[(size_t)t * NSUB * nch_gu + (pc % NSUB) * nch_gu + pc / NSUB] =
+                permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
         }
         cs = cons_sum_int(cs, C.redi);
         if (ctid == 0) {
@@ -267,21 +440,46 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         }
     }
     named_sync(kDecBar, kDecCons);
+    if (ctid == 0) DEC_TRACE(1);
+    // single-token decode with the production shape: the lane's activation
+    // chunks stay in registers for every gate/up row
+    uint4 xr[NG > 0 ? NG : 1][NSUB];
+    if (TM == 1 && NG > 0) {
+#pragma unroll
+        for (int i = 0; i < (NG > 0 ? NG : 1); ++i)
+#pragma unroll
+            for (int sb = 0; sb < NSUB; ++sb) xr[i][sb] = xs[sb * nch_gu + lane + 32 * i];
+    }
 
-    uint32_t u = 0;  // unit counter, identical sequence to the producer's
+    // unit index (identical sequence to the producer's) and its ring slot and
+    // phase, advanced without divisions; unit u belongs to group u & 1
+    uint32_t u = 0;
+    int cs_slot = 0;
+    uint32_t cs_phase = 0;
+    unsigned long long t_full = 0;  // time thread 0 spent waiting for data (traced)
+    auto next_unit = [&]() {
+        ++u;
+        if (++cs_slot == nslot) {
+            cs_slot = 0;
+            cs_phase ^= 1u;
+        }
+    };
     auto wait_full = [&]() -> const uint8_t* {
-        const int s = u % nslot;
-        mbar_wait_bounded(&C.full[s], (u / nslot) & 1, hdr, 200 + s);
-        return ring + (size_t)s * slot_bytes;
+        const unsigned long long t0 = (trace && ctid == 0) ? global_timer_ns() : 0;
+        mbar_wait_bounded(&C.full[cs_slot], cs_phase, hdr, 200 + cs_slot);
+        if (trace && ctid == 0) t_full += global_timer_ns() - t0;
+        return ring + (size_t)cs_slot * slot_bytes;
     };
     auto release = [&]() {
         __syncwarp();
-        if (lane == 0) mbar_arrive(&C.empty[u % nslot]);
-        ++u;
+        if (lane == 0) mbar_arrive(&C.empty[cs_slot]);
     };
+    const bool mine_even = grp == 0;
+    auto mine = [&]() { return ((u & 1) == 0) == mine_even; };
 
     // ---- 2. router units ----
-    for (int ru = 0; ru < n_router_units; ++ru) {
+    for (int ru = 0; ru < n_router_units; ++ru, next_unit()) {
+        if (!mine()) continue;
         const int rows = min(pl.rr, n_my_router - ru * pl.rr);
         const float* wrow = reinterpret_cast<const float*>(wait_full());
         float acc[2][TM];
@@ -289,7 +487,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         for (int i = 0; i < 2; ++i)
 #pragma unroll
             for (int t = 0; t < TM; ++t) acc[i][t] = 0.0f;
-        for (int v = ctid; v < d / 4; v += kDecCons) {
+        for (int v = gtid; v < d / 4; v += kDecGrp) {
             float4 wv[2];
             wv[0] = reinterpret_cast<const float4*>(wrow)[v];
             wv[1] = rows > 1 ? reinterpret_cast<const float4*>(wrow + d)[v] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -312,23 +510,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
 #pragma unroll
             for (int t = 0; t < TM; ++t) {
                 const float v = warp_sum(acc[i][t]);
-                if (lane == 0) C.part[warp][i * TM + t] = v;
+                if (lane == 0) C.part[grp][gw][i * TM + t] = v;
             }
-        named_sync(kDecBar, kDecCons);
-        if (ctid < rows * T) {
-            const int i = ctid / T, t = ctid % T;
+        named_sync(2 + grp, kDecGrp);
+        if (gtid < rows * T) {
+            const int i = gtid / T, t = gtid % T;
             float v = 0.0f;
 #pragma unroll
-            for (int w = 0; w < kDecWarps; ++w) v += C.part[w][i * TM + t];
+            for (int w = 0; w < kDecWarps; ++w) v += C.part[grp][w][i * TM + t];
             const int e = c + (ru * pl.rr + i) * G;
             p.ws.logits[(size_t)t * E + e] = v;
         }
-        named_sync(kDecBar, kDecCons);
+        named_sync(2 + grp, kDecGrp);
     }
     // arrive at the grid barrier (logits of this CTA published)
     __threadfence();
     named_sync(kDecBar, kDecCons);
     if (ctid == 0) {
+        DEC_TRACE(2);
         const unsigned ticket = atomicAdd(&hdr->b1_count, 1u);
         if (ticket == (unsigned)G - 1) {
             hdr->b1_count = 0u;
@@ -338,57 +537,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     }
 
     // ---- per-warp gate/up bookkeeping ----
-    int cur_task = -1, cur_cnt = 0;
+    int cur_task = -1, cur_cnt = 0, cur_n = 0;
+    int xoff[TM];    // staged-row offsets (uint4) of the current task's tokens
+    int t_asg[TM];   // their assignment ids
+    int t_cs[TM];    // their code sums
+    float t_sx[TM];  // their scales
     float amax[TM];
 #pragma unroll
-    for (int i = 0; i < TM; ++i) amax[i] = 0.0f;
-
-    auto requant = [&](int ti) {  // one warp: h of task ti -> hq, sh; publish
-        const int n = C.tasks[ti].y;
-        for (int i = 0; i < n; ++i) {
-            const int a = C.ttok[ti][i];
-            const float m = __uint_as_float(__ldcg(p.ws.amax + a));
-            const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-            const float* hrow = p.ws.h + (size_t)a * f;
-            int8_t* qrow = p.ws.hq + (size_t)a * f;
-            for (int cc = lane * 4; cc < f; cc += 128) {
-                const float4 hv = __ldcg(reinterpret_cast<const float4*>(hrow + cc));
-                char4 q = make_char4(0, 0, 0, 0);
-                if (m != 0.0f)
-                    q = make_char4((signed char)quant_code(hv.x, sh), (signed char)quant_code(hv.y, sh),
-                                   (signed char)quant_code(hv.z, sh), (signed char)quant_code(hv.w, sh));
-                *reinterpret_cast<char4*>(qrow + cc) = q;
-            }
-            __syncwarp();  // every lane has read amax[a]
-            if (lane == 0) {
-                p.ws.sh[a] = sh;
-                p.ws.amax[a] = 0u;  // ready for the next call
-            }
-        }
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) {
-            p.ws.task_ctr[ti] = 0u;
-            st_release_u32(p.ws.ready + ti, epoch + 1);
-        }
-    };
+    for (int i = 0; i < TM; ++i) {
+        amax[i] = 0.0f;
+        xoff[i] = 0;
+        t_asg[i] = 0;
+        t_cs[i] = 0;
+        t_sx[i] = 0.0f;
+    }
     auto flush_gu = [&]() {
         if (cur_task < 0 || cur_cnt == 0) return;
-        const int n = C.tasks[cur_task].y;
 #pragma unroll
         for (int i = 0; i < TM; ++i)
-            if (i < n && lane == i) atomicMax(p.ws.amax + C.ttok[cur_task][i], __float_as_uint(amax[i]));
+            if (i < cur_n && lane == i) atomicMax(amax_cur + t_asg[i], __float_as_uint(amax[i]));
         __threadfence();
         __syncwarp();
-        unsigned last = 0;
-        if (lane == 0) {
+        if (lane == 0) {  // the warp bringing the task's last rows publishes it
             const unsigned t0 = atomicAdd(p.ws.task_ctr + cur_task, (unsigned)cur_cnt);
-            last = t0 + cur_cnt == (unsigned)(pl.nu_gu * kDecWarps);
-        }
-        last = __shfl_sync(kFull, last, 0);
-        if (last) {
-            __threadfence();
-            requant(cur_task);
+            if (t0 + cur_cnt == (unsigned)(pl.nu_gu * kDecWarps)) {
+                p.ws.task_ctr[cur_task] = 0u;
+                __threadfence();
+                st_release_u32(p.ws.ready + cur_task, epoch + 1);
+            }
         }
         cur_cnt = 0;
 #pragma unroll
@@ -398,41 +574,76 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         if (ti != cur_task) {
             flush_gu();
             cur_task = ti;
+            cur_n = C.tasks[ti].y;
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+                if (i < cur_n) {
+                    t_asg[i] = C.ttok[ti][i];
+                    const int tok = t_asg[i] / S;
+                    xoff[i] = tok * NSUB * nch_gu;
+                    t_cs[i] = C.xcs[tok];
+                    t_sx[i] = C.sx[tok];
+                }
         }
         const uint8_t* slot = wait_full();
-        const int r = j * kDecWarps + warp;
-        const int4 tk = C.tasks[ti];
-        const int n = tk.y;
+        const int r = j * kDecWarps + gw;
+        const int n = cur_n;
         if (r < f) {
-            const uint8_t* grow = slot + (size_t)warp * rb_gu;
-            const uint8_t* urow = slot + (size_t)(kDecWarps + warp) * rb_gu;
+            const uint8_t* grow = slot + (size_t)gw * rb_gu;
+            const uint8_t* urow = slot + (size_t)(kDecWarps + gw) * rb_gu;
             int ag[TM], au[TM];
 #pragma unroll
             for (int i = 0; i < TM; ++i) ag[i] = au[i] = 0;
-            for (int cc = lane; cc < nch_gu; cc += 32) {
-                const uint4 wg = *reinterpret_cast<const uint4*>(grow + (size_t)cc * 16);
-                const uint4 wu = *reinterpret_cast<const uint4*>(urow + (size_t)cc * 16);
+            if constexpr (NG > 0) {
+                uint4 wg[NG], wu[NG];
 #pragma unroll
-                for (int i = 0; i < TM; ++i)
-                    if (i < n) {
-                        const uint4* xt = xs + (size_t)(C.ttok[ti][i] / S) * NSUB * nch_gu;
-                        ag[i] = dot_chunk<WB>(wg, xt, nch_gu, cc, ag[i]);
-                        au[i] = dot_chunk<WB>(wu, xt, nch_gu, cc, au[i]);
+                for (int i = 0; i < NG; ++i) {
+                    wg[i] = *reinterpret_cast<const uint4*>(grow + (size_t)(lane + 32 * i) * 16);
+                    wu[i] = *reinterpret_cast<const uint4*>(urow + (size_t)(lane + 32 * i) * 16);
+                }
+                if constexpr (TM == 1) {
+                    int g0 = 0, g1 = 0, u0 = 0, u1 = 0;
+#pragma unroll
+                    for (int i = 0; i < NG; ++i) {
+                        dot_chunk_regs<WB>(wg[i], xr[i], g0, g1);
+                        dot_chunk_regs<WB>(wu[i], xr[i], u0, u1);
                     }
+                    ag[0] = g0 + g1;
+                    au[0] = u0 + u1;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < NG; ++i)
+#pragma unroll
+                        for (int t = 0; t < TM; ++t)
+                            if (t < n) {
+                                ag[t] = dot_chunk<WB>(wg[i], xs + xoff[t], nch_gu, lane + 32 * i, ag[t]);
+                                au[t] = dot_chunk<WB>(wu[i], xs + xoff[t], nch_gu, lane + 32 * i, au[t]);
+                            }
+                }
+            } else {
+                for (int cc = lane; cc < nch_gu; cc += 32) {
+                    const uint4 wg = *reinterpret_cast<const uint4*>(grow + (size_t)cc * 16);
+                    const uint4 wu = *reinterpret_cast<const uint4*>(urow + (size_t)cc * 16);
+#pragma unroll
+                    for (int t = 0; t < TM; ++t)
+                        if (t < n) {
+                            ag[t] = dot_chunk<WB>(wg, xs + xoff[t], nch_gu, cc, ag[t]);
+                            au[t] = dot_chunk<WB>(wu, xs + xoff[t], nch_gu, cc, au[t]);
+                        }
+                }
             }
-            const float* sc = p.scales + (size_t)tk.x * p.scale_rows;
-            const float sg = __ldg(sc + r), su = __ldg(sc + f + r);
+            const float* ssc = reinterpret_cast<const float*>(slot + pl.wbytes);
+            const float sg = ssc[gw], su = ssc[kDecWarps + gw];
 #pragma unroll
             for (int i = 0; i < TM; ++i)
                 if (i < n) {
-                    const int a = C.ttok[ti][i], tok = a / S;
-                    const int Gv = __reduce_add_sync(kFull, ag[i]) - code_offset<WB>() * C.xcs[tok];
-                    const int Uv = __reduce_add_sync(kFull, au[i]) - code_offset<WB>() * C.xcs[tok];
+                    const int Gv = __reduce_add_sync(kFull, ag[i]) - code_offset<WB>() * t_cs[i];
+                    const int Uv = __reduce_add_sync(kFull, au[i]) - code_offset<WB>() * t_cs[i];
                     if (lane == i) {
-                        const float g = __fmul_rn((float)Gv, __fmul_rn(sg, C.sx[tok]));
-                        const float uu = __fmul_rn((float)Uv, __fmul_rn(su, C.sx[tok]));
+                        const float g = __fmul_rn((float)Gv, __fmul_rn(sg, t_sx[i]));
+                        const float uu = __fmul_rn((float)Uv, __fmul_rn(su, t_sx[i]));
                         const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), uu);
-                        p.ws.h[(size_t)a * f + r] = h;
+                        p.ws.h[(size_t)t_asg[i] * f + r] = h;
                         amax[i] = fmaxf(amax[i], fabsf(h));
                     }
                 }
@@ -442,24 +653,30 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     };
 
     // ---- 3. shared-expert gate/up units (no routing needed) ----
-    for (int i = 0; i < n_sh_units; ++i) {
-        if (i == 0) {  // the shared task's description, known before routing
-            if (ctid < T) C.ttok[0][ctid] = ctid * S + k;
-            if (ctid == 0) C.tasks[0] = make_int4(E, T, 0, 0);
-            named_sync(kDecBar, kDecCons);
-        }
-        gu_unit(0, c + i * G);
+    if (n_sh_units > 0) {  // the shared task's description, known before routing
+        if (ctid < T) C.ttok[0][ctid] = ctid * S + k;
+        if (ctid == 0) C.tasks[0] = make_int4(E, T, 0, 0);
+        named_sync(kDecBar, kDecCons);
     }
+    for (int i = 0; i < n_sh_units; ++i, next_unit())
+        if (mine()) gu_unit(0, c + i * G);
 
+    if (ctid == 0) DEC_TRACE(3);
     // ---- 4. grid barrier, then every CTA derives the routing ----
     if (ctid == 0) flag_wait_bounded(&hdr->b1_gen, epoch + 1, hdr, 300);
     named_sync(kDecBar, kDecCons);
+    if (ctid == 0) DEC_TRACE(4);
     if (c == 0 && ctid == 0) hdr->epoch = epoch + 1;
+    for (int i = c * kDecCons + ctid; i < p.a_cap; i += G * kDecCons) amax_nxt[i] = 0u;
     if (warp < T) {
-        float* scr = reinterpret_cast<float*>(hsb) + (size_t)warp * 2 * E;
         int my_e;
         float my_w;
-        topk_warp(p.ws.logits + (size_t)warp * E, p.bias, E, k, p.routed_scale, scr, scr + E, my_e, my_w);
+        if (E <= kDecBiasCache) {
+            topk_warp_small(p.ws.logits + (size_t)warp * E, C.bias_s, E, k, p.routed_scale, my_e, my_w);
+        } else {
+            float* scr = reinterpret_cast<float*>(hsb) + (size_t)warp * 2 * E;
+            topk_warp(p.ws.logits + (size_t)warp * E, p.bias, E, k, p.routed_scale, scr, scr + E, my_e, my_w);
+        }
         if (lane < k) {
             C.idx[warp][lane] = my_e;
             C.w[warp][lane] = my_w;
@@ -474,110 +691,192 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     named_sync(kDecBar, kDecCons);
     // bucket: sort the T*k assignments by (expert, token, slot); one task per expert
     const int A = T * k;
-    if (ctid < A) {
-        const int ea = C.idx[ctid / k][ctid % k];
-        int pos = 0;
-        for (int a2 = 0; a2 < A; ++a2) {
-            const int e2 = C.idx[a2 / k][a2 % k];
-            pos += (e2 < ea) || (e2 == ea && a2 < ctid);
+    if (T == 1) {  // one token: the k experts, each a task with that token, by ascending expert
+        if (warp == 0) {
+            const int e = lane < k ? C.idx[0][lane] : 0x7fffffff;
+            int rank = 0;
+            for (int j = 0; j < k; ++j) rank += __shfl_sync(kFull, e, j) < e;
+            if (lane < k) {
+                C.ttok[HS + rank][0] = lane;  // assignment id: token 0, slot lane
+                C.tasks[HS + rank] = make_int4(e, 1, 0, 0);
+            }
+            if (HS && lane == 0) {
+                C.ttok[0][0] = k;
+                C.tasks[0] = make_int4(E, 1, 0, 0);
+            }
+            if (lane == 0) C.n_tasks = HS + k;
         }
+    } else if (ctid < A) {
+        const int ea = C.idx[ctid / k][ctid % k];
+        int pos = 0, a2 = 0;
+        for (int t2 = 0; t2 < T; ++t2)
+            for (int j2 = 0; j2 < k; ++j2, ++a2) {
+                const int e2 = C.idx[t2][j2];
+                pos += (e2 < ea) || (e2 == ea && a2 < ctid);
+            }
         C.sorted[pos] = ctid;
+        C.sorted_e[pos] = ea;
     }
-    if (HS && ctid < T) C.ttok[0][ctid] = ctid * S + k;
-    if (HS && ctid == 0) C.tasks[0] = make_int4(E, T, 0, 0);
+    if (T > 1 && HS && ctid < T) C.ttok[0][ctid] = ctid * S + k;
+    if (T > 1 && HS && ctid == 0) C.tasks[0] = make_int4(E, T, 0, 0);
     named_sync(kDecBar, kDecCons);
-    if (ctid < A) {
+    if (T > 1 && ctid < A) {
         const int a = C.sorted[ctid];
-        const int ea = C.idx[a / k][a % k];
+        const int ea = C.sorted_e[ctid];
         int ti = -1, rank = 0, n = 0;
         for (int q = 0; q <= ctid; ++q) {
-            const int aq = C.sorted[q];
-            const int eq = C.idx[aq / k][aq % k];
-            const int ep = q == 0 ? -1 : C.idx[C.sorted[q - 1] / k][C.sorted[q - 1] % k];
-            ti += eq != ep;
+            const int eq = C.sorted_e[q];
+            ti += eq != (q == 0 ? -1 : C.sorted_e[q - 1]);
             rank += (eq == ea) && q < ctid;
         }
-        for (int q = 0; q < A; ++q) {
-            const int aq = C.sorted[q];
-            n += C.idx[aq / k][aq % k] == ea;
-        }
+        for (int q = 0; q < A; ++q) n += C.sorted_e[q] == ea;
         C.ttok[HS + ti][rank] = (a / k) * S + (a % k);
         if (rank == 0) C.tasks[HS + ti] = make_int4(ea, n, 0, 0);
         if (ctid == A - 1) C.n_tasks = HS + ti + 1;
     }
     named_sync(kDecBar, kDecCons);
-    if (ctid == 0) mbar_arrive(&C.route_ready);  // the producer may issue routed rows
+    if (ctid == 0) {
+        mbar_arrive(&C.route_ready);  // the producer may issue routed rows
+        DEC_TRACE(5);
+    }
     const int n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
 
     // ---- 5. routed gate/up units ----
     {
         const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
-        for (long long g = c * Nr / G; g < (c + 1) * Nr / G; ++g)
-            gu_unit(HS + (int)(g / pl.nu_gu), (int)(g % pl.nu_gu));
+        const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
+        int ti = HS + (int)(lo / pl.nu_gu), j = (int)(lo % pl.nu_gu);
+        for (long long g = lo; g < hi; ++g, next_unit()) {
+            if (mine()) gu_unit(ti, j);
+            if (++j == pl.nu_gu) {
+                j = 0;
+                ++ti;
+            }
+        }
         flush_gu();
     }
+    if (ctid == 0) DEC_TRACE(6);
 
-    // ---- 6. down units + combine ----
+    // ---- 6. down units ----
+    uint8_t* hsg = hsb + (size_t)grp * hs_grp;  // this group's staged h codes
+    uint4 hr[ND > 0 ? ND : 1][NSUB];             // single token: the lane's h chunks
     const long long Nd = (long long)n_tasks * pl.nu_dn;
-    for (long long g = c * Nd / G; g < (c + 1) * Nd / G; ++g) {
-        const int ti = (int)(g / pl.nu_dn), j = (int)(g % pl.nu_dn);
-        const int4 tk = C.tasks[ti];
-        const int n = tk.y;
-        if (ti != C.hq_task) {  // stage this task's h codes (all consumer warps agree on ti)
-            named_sync(kDecBar, kDecCons);
-            if (ctid == 0) flag_wait_bounded(p.ws.ready + ti, epoch + 1, hdr, 400);
-            named_sync(kDecBar, kDecCons);
+    const long long dlo = c * Nd / G, dhi = (c + 1) * Nd / G;
+    int dti = (int)(dlo / pl.nu_dn), dj = (int)(dlo % pl.nu_dn);
+    for (long long g = dlo; g < dhi; ++g, next_unit()) {
+        const int ti = dti, j = dj;
+        if (++dj == pl.nu_dn) {
+            dj = 0;
+            ++dti;
+        }
+        if (!mine()) continue;
+        const int n = C.tasks[ti].y;
+        if (ti != C.hq_task[grp]) {  // requantise and stage this task's h (the whole group agrees on ti)
+            named_sync(2 + grp, kDecGrp);
+            if (gtid == 0) flag_wait_bounded(p.ws.ready + ti, epoch + 1, hdr, 400);
+            named_sync(2 + grp, kDecGrp);
             for (int i = 0; i < n; ++i) {
                 const int a = C.ttok[ti][i];
-                int cs = stage_row<WB>(p.ws.hq + (size_t)a * f, f,
-                                       reinterpret_cast<uint4*>(hsb) + (size_t)i * NSUB * nch_dn);
-                cs = cons_sum_int(cs, C.redi);
-                if (ctid == 0) {
-                    C.hcs[i] = cs;
-                    C.hsh[i] = __ldcg(p.ws.sh + a);
+                const float m = __uint_as_float(__ldcg(amax_cur + a));
+                const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+                const float* hrow = p.ws.h + (size_t)a * f;
+                uint4* hst = reinterpret_cast<uint4*>(hsg) + (size_t)i * NSUB * nch_dn;
+                int cs = 0;
+                for (int pc = gtid; pc < f / 16; pc += kDecGrp) {
+                    unsigned wds[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 hv = __ldcg(reinterpret_cast<const float4*>(hrow + pc * 16 + 4 * q4));
+                        const float hs4[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int code = m == 0.0f ? 0 : quant_code(hs4[q], sh);
+                            cs += code;
+                            wds[q4] |= ((unsigned)code & 0xFFu) << (8 * q);
+                        }
+                    }
+                    hst[(pc % NSUB) * nch_dn + pc / NSUB] = permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
+                }
+                cs = grp_sum_int(cs, C.redi, grp);
+                if (gtid == 0) {
+                    C.hcs[grp][i] = cs;
+                    C.hsh[grp][i] = sh;
                 }
             }
-            if (ctid == 0) C.hq_task = ti;
-            named_sync(kDecBar, kDecCons);
+            if (gtid == 0) {
+                if (C.hq_task[0] < 0 && C.hq_task[1] < 0) DEC_TRACE(7);
+                C.hq_task[grp] = ti;
+            }
+            named_sync(2 + grp, kDecGrp);
+            if constexpr (TM == 1 && ND > 0) {
+#pragma unroll
+                for (int i = 0; i < ND; ++i)
+#pragma unroll
+                    for (int sb = 0; sb < NSUB; ++sb) hr[i][sb] = reinterpret_cast<const uint4*>(hsg)[sb * nch_dn + lane + 32 * i];
+            }
         }
         const uint8_t* slot = wait_full();
-        const float* sd = p.scales + (size_t)tk.x * p.scale_rows + 2 * f;
-        for (int q = 0; q < pl.rd / kDecWarps; ++q) {
-            const int rl = q * kDecWarps + warp, r = j * pl.rd + rl;
+        const float* sd = reinterpret_cast<const float*>(slot + pl.wbytes);  // this unit's row scales
+        const int nq = pl.rd / kDecWarps;
+        for (int q = 0; q < nq; ++q) {
+            const int rl = q * kDecWarps + gw, r = j * pl.rd + rl;
             if (r >= d) break;
             const uint8_t* wrow = slot + (size_t)rl * rb_dn;
             int acc[TM];
 #pragma unroll
             for (int i = 0; i < TM; ++i) acc[i] = 0;
-            for (int cc = lane; cc < nch_dn; cc += 32) {
-                const uint4 wv = *reinterpret_cast<const uint4*>(wrow + (size_t)cc * 16);
+            if constexpr (TM == 1 && ND > 0) {
+                int a0 = 0, a1 = 0;
 #pragma unroll
-                for (int i = 0; i < TM; ++i)
-                    if (i < n) acc[i] = dot_chunk<WB>(wv, reinterpret_cast<const uint4*>(hsb) + (size_t)i * NSUB * nch_dn,
-                                                      nch_dn, cc, acc[i]);
+                for (int i = 0; i < ND; ++i)
+                    dot_chunk_regs<WB>(*reinterpret_cast<const uint4*>(wrow + (size_t)(lane + 32 * i) * 16), hr[i], a0,
+                                       a1);
+                acc[0] = a0 + a1;
+            } else {
+                for (int cc = lane; cc < nch_dn; cc += 32) {
+                    const uint4 wv = *reinterpret_cast<const uint4*>(wrow + (size_t)cc * 16);
+#pragma unroll
+                    for (int i = 0; i < TM; ++i)
+                        if (i < n)
+                            acc[i] = dot_chunk<WB>(wv, reinterpret_cast<const uint4*>(hsg) + (size_t)i * NSUB * nch_dn,
+                                                   nch_dn, cc, acc[i]);
+                }
             }
-            const float sdr = __ldg(sd + r);
+            const float sdr = sd[rl];
 #pragma unroll
             for (int i = 0; i < TM; ++i)
                 if (i < n) {
-                    const int D = __reduce_add_sync(kFull, acc[i]) - code_offset<WB>() * C.hcs[i];
+                    const int D = __reduce_add_sync(kFull, acc[i]) - code_offset<WB>() * C.hcs[grp][i];
                     if (lane == i) {
                         const int a = C.ttok[ti][i];
-                        p.ws.ybuf[(size_t)a * d + r] = __fmul_rn((float)D, __fmul_rn(sdr, C.hsh[i]));
+                        p.ws.ybuf[(size_t)a * d + r] = __fmul_rn((float)D, __fmul_rn(sdr, C.hsh[grp][i]));
                     }
                 }
         }
         release();
-        // row block j: the warp bringing its last contribution combines it
-        __threadfence();
-        __syncwarp();
-        unsigned last = 0;
-        if (lane == 0) last = atomicAdd(p.ws.rb_ctr + j, 1u) == (unsigned)(n_tasks * kDecWarps - 1);
-        last = __shfl_sync(kFull, last, 0);
-        if (last) {
-            __threadfence();
-            const int r0 = j * pl.rd, rows = min(pl.rd, d - r0);
-            for (int i = lane; i < T * rows; i += 32) {
+    }
+
+    // ---- 7. sign off this CTA's row blocks; the CTA completing one combines it ----
+    named_sync(kDecBar, kDecCons);  // every down output of this CTA is written
+    for (long long base = dlo; base < dhi; base += kDecCons) {
+        if (ctid == 0) C.n_last = 0;
+        named_sync(kDecBar, kDecCons);
+        const long long g = base + ctid;
+        if (g < dhi) {
+            const int rb = (int)(g % pl.nu_dn);
+            __threadfence();  // release: the CTA's stores (ordered by the barrier) before the arrival
+            if (atomicAdd(p.ws.rb_ctr + rb, 1u) == (unsigned)(n_tasks - 1)) {
+                p.ws.rb_ctr[rb] = 0u;
+                C.last_rb[atomicAdd(&C.n_last, 1)] = rb;
+            }
+        }
+        named_sync(kDecBar, kDecCons);
+        const int n_last = C.n_last;
+        if (n_last > 0) __threadfence();  // acquire: the other CTAs' down outputs
+        for (int li = 0; li < n_last; ++li) {
+            const int rb = C.last_rb[li];
+            const int r0 = rb * pl.rd, rows = min(pl.rd, d - r0);
+            for (int i = ctid; i < T * rows; i += kDecCons) {
                 const int t = i / rows, r = r0 + i % rows;
                 float o = 0.0f;
                 for (int jj = 0; jj < k; ++jj)
@@ -586,9 +885,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 float* dst = p.out + (size_t)t * d + r;
                 *dst = p.accumulate ? *dst + o : o;
             }
-            if (lane == 0) p.ws.rb_ctr[j] = 0u;
         }
+        named_sync(kDecBar, kDecCons);
     }
+    if (ctid == 0) {
+        DEC_TRACE(8);
+        if (trace) trace[9] = t_full;
+    }
+#undef DEC_TRACE
 }
 
 }  // namespace moe

@@ -13,20 +13,30 @@ bool decode_plan(const Dims& m, DecPlan* pl) {
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
     const int rb_gu = m.d * m.wb / 8, rb_dn = m.f * m.wb / 8;
-    int slot = std::max(2 * kDecWarps * rb_gu, kDecWarps * rb_dn);
-    slot = std::max(slot, m.d * 4);
-    slot = (int)align_up((size_t)slot, 128);
+    if (m.d > 16 * kDecCons) return false;  // the quantiser holds one 16-value piece per consumer thread
+    int wbytes = std::max(2 * kDecWarps * rb_gu, kDecWarps * rb_dn);
+    wbytes = std::max(wbytes, m.d * 4);
+    wbytes = (int)align_up((size_t)wbytes, 128);
     DecPlan q{};
+    q.wbytes = wbytes;
+    q.rr = std::min(2, wbytes / (m.d * 4));
+    q.rd = (wbytes / rb_dn) / kDecWarps * kDecWarps;
+    // row scales of a unit follow its weights: 2 x 8 (gate/up) or rd (down) floats
+    const int slot = (int)align_up((size_t)wbytes + 4 * std::max(2 * kDecWarps, q.rd), 128);
     q.slot_bytes = slot;
-    q.rr = std::min(2, slot / (m.d * 4));
-    q.rd = (slot / rb_dn) / kDecWarps * kDecWarps;
     q.nu_gu = (m.f + kDecWarps - 1) / kDecWarps;
     q.nu_dn = (m.d + q.rd - 1) / q.rd;
     const int ctl = (int)align_up(sizeof(DecCtl), 128);
     const int xs = (int)align_up((size_t)m.T * m.d, 128);
-    const int hs = (int)align_up(std::max((size_t)m.T * m.f, (size_t)8 * m.T * m.E), 128);
+    q.hs_grp_bytes = (int)align_up((size_t)m.T * m.f, 128);
+    // h staging of both consumer groups; the same bytes serve the top-k scratch
+    const int hs = (int)align_up(std::max((size_t)kDecGroups * q.hs_grp_bytes, (size_t)8 * m.T * m.E), 128);
     const int room = optin - ctl - xs - hs - 1024;  // keep 1 KB for static shared memory
-    q.nslot = std::min(kDecMaxSlots, room / slot);
+    // an even slot count: the two consumer groups take alternate units, so
+    // each group then owns the slots of its parity and waits on consecutive
+    // phases of each (an odd count would let a group reach a slot two rounds
+    // ahead, where a parity wait cannot tell the phases apart)
+    q.nslot = std::min(kDecMaxSlots, room / slot) / 2 * 2;
     if (q.nslot < 2) return false;
     q.xs_off = ctl;
     q.hs_off = ctl + xs;
@@ -36,9 +46,9 @@ bool decode_plan(const Dims& m, DecPlan* pl) {
     return true;
 }
 
-template <int WB, int TM, typename XT>
+template <int WB, int TM, int NG, int ND, typename XT>
 static cudaError_t go(const Params& p, const DecPlan& pl, const void* x, cudaStream_t s) {
-    auto fn = k_decode<WB, TM, XT>;
+    auto fn = k_decode<WB, TM, NG, ND, XT>;
     cudaError_t e = allow_smem((const void*)fn, pl.smem_bytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
@@ -52,19 +62,30 @@ static cudaError_t go(const Params& p, const DecPlan& pl, const void* x, cudaStr
     return cudaLaunchCooperativeKernel((const void*)fn, dim3(sms), dim3(kDecThreads), args, pl.smem_bytes, s);
 }
 
-template <int WB, typename XT>
+template <int WB, int NG, int ND, typename XT>
 static cudaError_t by_t(const Params& p, const DecPlan& pl, const void* x, cudaStream_t s) {
     const int T = p.m.T;
-    if (T <= 1) return go<WB, 1, XT>(p, pl, x, s);
-    if (T <= 2) return go<WB, 2, XT>(p, pl, x, s);
-    if (T <= 4) return go<WB, 4, XT>(p, pl, x, s);
-    return go<WB, 8, XT>(p, pl, x, s);
+    if (T <= 1) return go<WB, 1, NG, ND, XT>(p, pl, x, s);
+    if (T <= 2) return go<WB, 2, NG, ND, XT>(p, pl, x, s);
+    if (T <= 4) return go<WB, 4, NG, ND, XT>(p, pl, x, s);
+    return go<WB, 8, NG, ND, XT>(p, pl, x, s);
+}
+
+// Fully unrolled rows for the GLM-5.2 expert shape (d = 6144, f = 2048):
+// 6 (int4) or 3 (int2) 16-byte chunks per lane of a gate/up row, 2 or 1 of a
+// down row; any other shape takes the runtime loop.
+template <int WB, typename XT>
+static cudaError_t by_shape(const Params& p, const DecPlan& pl, const void* x, cudaStream_t s) {
+    const int nch_gu = p.m.d * WB / 8 / 16, nch_dn = p.m.f * WB / 8 / 16;
+    constexpr int NG = WB == 4 ? 6 : 3, ND = WB == 4 ? 2 : 1;
+    if (nch_gu == 32 * NG && nch_dn == 32 * ND) return by_t<WB, NG, ND, XT>(p, pl, x, s);
+    return by_t<WB, 0, 0, XT>(p, pl, x, s);
 }
 
 cudaError_t launch_decode(const Params& p, const DecPlan& pl, const void* x, bool bf16, cudaStream_t s) {
     if (p.m.wb == 4)
-        return bf16 ? by_t<4, __nv_bfloat16>(p, pl, x, s) : by_t<4, float>(p, pl, x, s);
-    return bf16 ? by_t<2, __nv_bfloat16>(p, pl, x, s) : by_t<2, float>(p, pl, x, s);
+        return bf16 ? by_shape<4, __nv_bfloat16>(p, pl, x, s) : by_shape<4, float>(p, pl, x, s);
+    return bf16 ? by_shape<2, __nv_bfloat16>(p, pl, x, s) : by_shape<2, float>(p, pl, x, s);
 }
 
 }  // namespace moe

@@ -151,13 +151,22 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *  path: MOE_PATH_AUTO (0), MOE_PATH_MULTI (1: separate routing, gate/up and
  *        down kernels) or MOE_PATH_DECODE (2: one persistent kernel for
  *        T <= 8; MOE_EINVAL if the shape does not fit it).
- *  n_launches: set to the number of kernels the call launched. */
+ *  n_launches: set to the number of kernels the call launched.
+ *  trace: optional DEVICE buffer of (number of SMs) x 16 uint64 that the
+ *         single-launch decode path fills with per-CTA global-timer stamps
+ *         (ns) at its phase boundaries: [0] start, [1] tokens quantised,
+ *         [2] router rows done, [3] shared-expert gate/up done, [4] grid
+ *         barrier passed, [5] routing derived, [6] routed gate/up done,
+ *         [7] first down staging ready, [8] down done; producer: [12] rows
+ *         known before routing issued, [13] routing received, [14] all rows
+ *         issued, [15] all copies landed.  Untouched entries are left as is. */
 enum { MOE_PATH_AUTO = 0, MOE_PATH_MULTI = 1, MOE_PATH_DECODE = 2 };
 typedef struct {
     void* events[4];
     int32_t path;
     int32_t n_launches;
-    int32_t reserved[6];
+    void* trace;
+    int32_t reserved[4];
 } moe_layer_opts;
 
 /* moe_layer with options (opts may be NULL, then identical to moe_layer). */
