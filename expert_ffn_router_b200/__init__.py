@@ -75,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "moe_workspace_init": (I32, [P, SZ, P]),
         "moe_quantize": (I32, [C, P, I32, I32, P, P, P]),
         "moe_route": (I32, [C, P, I32, I32, P, P, P, P, P, SZ, P]),
+        "moe_route_static": (I32, [C, P, I32, I32, P, P, P, P, P]),
         "moe_expert_ffn": (I32, [C, PL, I32, P, P, I32, P, P, P, P, P, P, SZ, P]),
         "moe_expert_down": (I32, [C, PL, I32, P, P, I32, P, P, P, SZ, P]),
         "moe_layer": (I32, [C, PL, P, P, P, I32, I32, P, I32, P, P, P, SZ, P]),
@@ -174,6 +175,20 @@ def moe_route(cfg: MoeConfig, x: torch.Tensor, w_router: torch.Tensor, bias: tor
                          _ptr(topk_idx, torch.int32, T * cfg.top_k, "topk_idx"),
                          _ptr(topk_w, torch.float32, T * cfg.top_k, "topk_w"),
                          _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream)), "moe_route")
+
+
+def moe_route_static(cfg: MoeConfig, x: torch.Tensor, w_router: torch.Tensor, bias: torch.Tensor,
+                     topk_idx: torch.Tensor, topk_w: torch.Tensor, stream=None):
+    """moe_route without a workspace, for callers that cannot allocate device
+    memory on their call path; its scratch is a fixed array inside libmoe.so.
+    Up to 8 tokens per call; calls that overlap on the GPU race."""
+    T = x.shape[0]
+    _check(lib.moe_route_static(ctypes.byref(cfg), _ptr(x, name="x"), _xdtype(x), T,
+                                _ptr(w_router, torch.float32, cfg.n_experts * cfg.d, "w_router"),
+                                _ptr(bias, torch.float32, cfg.n_experts, "bias"),
+                                _ptr(topk_idx, torch.int32, T * cfg.top_k, "topk_idx"),
+                                _ptr(topk_w, torch.float32, T * cfg.top_k, "topk_w"), _stream(stream)),
+           "moe_route_static")
 
 
 def moe_expert_ffn(cfg: MoeConfig, pool: MoePool, expert: int, xq: torch.Tensor, sx: torch.Tensor,

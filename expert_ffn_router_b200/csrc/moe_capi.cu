@@ -19,7 +19,7 @@ namespace moe {
 
 static thread_local std::string g_last_error;
 
-static moe_status fail(moe_status st, const std::string& msg) {
+moe_status fail(moe_status st, const std::string& msg) {
     g_last_error = msg;
     return st;
 }
@@ -101,7 +101,7 @@ ExpertTiling expert_tiling(int d, int f, int wb) {
 // ---------------------------------------------------------------------------
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-static moe_status check_cfg(const moe_config* c) {
+moe_status check_cfg(const moe_config* c) {
     if (!c) return fail(MOE_EINVAL, "cfg is NULL");
     if (c->d <= 0 || c->f <= 0 || c->d > 8192 || c->f > 8192)
         return fail(MOE_EINVAL, "d and f must be in [1, 8192]");
@@ -116,7 +116,7 @@ static moe_status check_cfg(const moe_config* c) {
     return MOE_OK;
 }
 
-static moe_status check_ptr(const void* p, const char* name, bool nullable = false) {
+moe_status check_ptr(const void* p, const char* name, bool nullable) {
     if (!p) return nullable ? MOE_OK : fail(MOE_EINVAL, std::string(name) + " is NULL");
     if (!aligned16(p)) return fail(MOE_EALIGN, std::string(name) + " is not 16-byte aligned");
     return MOE_OK;
@@ -232,13 +232,12 @@ static cudaError_t launch_router(Params& p, const XT* x, int do_quant, int bucke
     return cudaSuccess;
 }
 
-static cudaError_t launch_router_any(Params& p, const void* x, moe_dtype dt, int do_quant, int bucket,
-                                     cudaStream_t s) {
+cudaError_t launch_router_any(Params& p, const void* x, moe_dtype dt, int do_quant, int bucket, cudaStream_t s) {
     if (dt == MOE_BF16) return launch_router(p, static_cast<const __nv_bfloat16*>(x), do_quant, bucket, s);
     return launch_router(p, static_cast<const float*>(x), do_quant, bucket, s);
 }
 
-static moe_status check_dtype(moe_dtype dt) {
+moe_status check_dtype(moe_dtype dt) {
     return (dt == MOE_F32 || dt == MOE_BF16) ? MOE_OK : fail(MOE_EINVAL, "dtype must be MOE_F32 or MOE_BF16");
 }
 

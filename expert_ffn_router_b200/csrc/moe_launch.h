@@ -3,6 +3,8 @@
 
 #include <cuda_runtime.h>
 
+#include <string>
+
 #include "moe_common.cuh"
 
 namespace moe {
@@ -27,6 +29,14 @@ bool decode_plan(const Dims& m, DecPlan* pl);
 cudaError_t launch_decode(const Params& p, const DecPlan& pl, const void* x, bool bf16, cudaStream_t s);
 
 cudaError_t launch_gate_up(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s);
+
+// Router launch sequence (a0 + a1 (+ a2)) and the host-side checks the entry
+// points share (moe_capi.cu).
+cudaError_t launch_router_any(Params& p, const void* x, moe_dtype dt, int do_quant, int bucket, cudaStream_t s);
+moe_status fail(moe_status st, const std::string& msg);
+moe_status check_cfg(const moe_config* c);
+moe_status check_ptr(const void* p, const char* name, bool nullable = false);
+moe_status check_dtype(moe_dtype dt);
 cudaError_t launch_down(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s);
 
 }  // namespace moe

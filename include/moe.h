@@ -115,6 +115,27 @@ MOE_API moe_status moe_route(const moe_config* cfg, const void* x, moe_dtype dty
                      const float* w_router, const float* bias, int32_t* topk_idx, float* topk_w,
                      void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* The router of moe_route for callers that cannot provide a workspace.
+ * The Colibri pages have no counterpart for this entry point: it exists for
+ * callers of this library that cannot allocate device memory on their call
+ * path -- a host framework that owns all device memory and forbids allocations
+ * after start-up, a serving loop that must not pay cudaMalloc's implicit device
+ * synchronisation, a plugin interface with no way to request scratch space.
+ * Same arguments and results as moe_route, without ws/ws_bytes.  Its scratch
+ * (64 KB) is a fixed array inside libmoe.so that every GPU loading the library
+ * keeps until the process exits; the call allocates nothing.
+ *  - Limits: T <= 8 tokens, n_experts <= 1024, top_k <= 32; larger requests
+ *    return MOE_EINVAL with a message naming the limit.
+ *  - The first call on each device looks up that array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call, on every stream, shares the one array: calls whose work
+ *    overlaps on the GPU race and give undefined results.  Each call clears
+ *    the control word it needs at its start. */
+MOE_API moe_status moe_route_static(const moe_config* cfg, const void* x, moe_dtype dtype, int32_t T,
+                                    const float* w_router, const float* bias, int32_t* topk_idx, float* topk_w,
+                                    moe_stream_t stream);
+
 /* One expert over T tokens (steps a3 + a4): expert in [0, E) is a routed
  * expert, -1 the shared one.  xq int8 [T][d], sx fp32 [T] -> y fp32 [T][d]
  * (overwritten).  Optional debug outputs (NULL to skip): dbg_acc_gu int32
