@@ -112,16 +112,17 @@ class Clocks:
 # ---------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_decode_timer(wl, seed, token_sets):
-    """Prepare the oracle on the decode workload: route every token once,
+def oracle_decode_timer(wl, seed, token_sets, max_tokens=None):
+    """Prepare the oracle on the workload: route every sampled token once,
     generate the selected experts' blobs, and return a function that runs the
-    oracle layer on one token (timed by the caller)."""
+    oracle layer on one token set (at most max_tokens of its tokens; timed by
+    the caller)."""
     import numpy as np
 
     import oracle as O
     import workloads as W
     L = W.layer(wl, seed, 0)
-    xs = [W.tokens(wl, seed, s).float().numpy() for s in token_sets]
+    xs = [W.tokens(wl, seed, s).float().numpy()[:max_tokens] for s in token_sets]
     need = {wl.n_experts} if wl.has_shared else set()
     for x in xs:
         idx, _ = O.route(x, L.w_router, L.bias, wl.top_k, wl.routed_scale)
@@ -141,17 +142,22 @@ def oracle_decode_timer(wl, seed, token_sets):
 
 
 def cpu_baseline(wl, budget_s):
+    """The oracle layer on a bounded sample: up to 16 single-token sets, or 4
+    sets of at most 4 tokens for batched workloads (the oracle's per-token
+    cost of the layer does not depend on T)."""
     import oracle as O
-    run = oracle_decode_timer(wl, 0, list(range(16)))
+    per = min(wl.T, 4)
+    n_sets = 16 if per == 1 else 4  # bounds the experts generated on the host
+    run = oracle_decode_timer(wl, 0, list(range(n_sets)), max_tokens=per)
     n, t0 = 0, time.perf_counter()
     while True:
         run(n)
         n += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or n >= 16:
+        if el >= budget_s or n >= n_sets:
             break
-    return {"value": n * wl.T / el, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
-            "sample": f"{n} tokens of {wl.name} (T={wl.T} per token, full layer), {el:.1f} s of CPU work"}
+    return {"value": n * per / el, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"{n} calls of {per} token(s) of {wl.name}, full layer, {el:.1f} s of CPU work"}
 
 
 def reference_arm(args, wl):
@@ -336,7 +342,8 @@ def gpu_arm(args, wl):
                "h2d_bytes_per_step": T * wl.d * toks.element_size(), "d2h_bytes_per_step": T * wl.d * 4,
                "api": "expert_ffn_router_b200.moe_layer (libmoe.so moe_layer), pinned host buffers"}
 
-    single = opts[0].n_launches == 1
+    ran = opts[0].path_ran
+    single = ran == M.MOE_PATH_DECODE
     router_bytes = wl.n_experts * wl.d * 4
     if args.trace and rank == 0:
         write_trace(args.trace, M, cfg, pool, dl, xbuf, out, ws, dev, flush_l2)
@@ -346,8 +353,8 @@ def gpu_arm(args, wl):
             kname = "k_decode"
             k_avg_s = statistics.mean(step_ms) / 1e3
             k_alg = statistics.mean(u * (gu_bytes_e + dn_bytes_e) for u in uniq) + router_bytes
-        else:
-            kname = "k_gate_up"
+        else:  # the gate/up kernel: every unique expert's gate and up rows once
+            kname = "k_tc<gate/up>" if ran == M.MOE_PATH_TC else "k_gate_up"
             k_avg_s = statistics.mean(gu_ms) / 1e3
             k_alg = statistics.mean(u * gu_bytes_e for u in uniq)
         achieved = k_alg / k_avg_s / 1e9
@@ -367,7 +374,8 @@ def gpu_arm(args, wl):
         value = world * K * T / (max_ms / 1e3)
         exp_gbs = exp_bytes / (total_ms / 1e3) / 1e9
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
+            "metric": METRIC if args.workload == 1 else f"MoE-layer tokens/s on {wl.name}; expert-weight HBM GB/s",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "i8*i4->i32" if wl.wbits == 4 else "i8*i2->i32", "data": "synthetic",
             "config": {"workload": wl.name, "T": T, "d": wl.d, "f": wl.f, "experts": wl.n_experts,
@@ -377,6 +385,7 @@ def gpu_arm(args, wl):
                        "parallelism": f"replicas{world}"},
             "expert_weight_gbs": exp_gbs, "expert_weight_frac_of_8tbs": exp_gbs / NOMINAL_HBM_GBS,
             "expert_weight_frac_of_measured": exp_gbs / hbm, "unique_experts_per_step": statistics.mean(uniq),
+            "path": {M.MOE_PATH_DECODE: "decode", M.MOE_PATH_MULTI: "multi", M.MOE_PATH_TC: "tensor_core"}.get(ran),
             "phase_ms": ({"layer_single_launch": statistics.mean(step_ms)} if single else
                          {"route": statistics.mean(route_ms), "gate_up": statistics.mean(gu_ms),
                           "down_combine": statistics.mean(dn_ms)}),

@@ -22,7 +22,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "moe.h")
 
 MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_ENOSPACE, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 MOE_F32, MOE_BF16 = 0, 1
-MOE_PATH_AUTO, MOE_PATH_MULTI, MOE_PATH_DECODE = 0, 1, 2
+MOE_PATH_AUTO, MOE_PATH_MULTI, MOE_PATH_DECODE, MOE_PATH_TC = 0, 1, 2, 3
 
 
 class MoeError(RuntimeError):
@@ -51,7 +51,7 @@ class MoeConfig(ctypes.Structure):
 
 class MoeLayerOpts(ctypes.Structure):
     _fields_ = [("events", ctypes.c_void_p * 4), ("path", ctypes.c_int32), ("n_launches", ctypes.c_int32),
-                ("trace", ctypes.c_void_p), ("reserved", ctypes.c_int32 * 4)]
+                ("trace", ctypes.c_void_p), ("path_ran", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
 
 
 class MoePool(ctypes.Structure):
@@ -134,7 +134,11 @@ def _xdtype(x: torch.Tensor) -> int:
 
 
 def make_pool(w: torch.Tensor, s: torch.Tensor) -> MoePool:
-    return MoePool(_ptr(w, torch.uint8, name="pool.w"), _ptr(s, torch.float32, name="pool.s"))
+    """The C struct over two device tensors; it keeps references to them, so
+    their memory stays allocated for as long as the struct is in use."""
+    pool = MoePool(_ptr(w, torch.uint8, name="pool.w"), _ptr(s, torch.float32, name="pool.s"))
+    pool._tensors = (w, s)
+    return pool
 
 
 # ---------------------------------------------------------------------------

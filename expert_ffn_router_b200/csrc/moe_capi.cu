@@ -136,7 +136,19 @@ static int pick_ch(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8; }
 
 static Dims layout_dims(const moe_config* c, size_t ws_bytes);
 
-static Params base_params(const moe_config* c, const Dims& m, void* ws, size_t ws_bytes) {
+// Default of moe_config.tc_min_tokens: calls with at least this many tokens
+// run the experts on the tensor-core path.
+constexpr int kTcDefaultMinTokens = 16;
+
+static bool use_tc(const moe_config* c, int T) {
+    const int thr = c->tc_min_tokens == 0 ? kTcDefaultMinTokens : c->tc_min_tokens;
+    return thr > 0 && T >= thr && tc_shape_ok(dims_of(c, T, c->top_k + c->has_shared));
+}
+
+// Bound on the tokens of one tensor-core task in a call of T tokens.
+static int tc_nt_max(int T) { return tc_npad(std::min(T, kTcNT)); }
+
+static Params base_params(const moe_config* c, const Dims& m, void* ws, size_t ws_bytes, bool tc = false) {
     Params p{};
     p.m = m;
     p.routed_scale = c->routed_scale;
@@ -148,6 +160,14 @@ static Params base_params(const moe_config* c, const Dims& m, void* ws, size_t w
     p.nrb3 = (c->f + p.rb3 - 1) / p.rb3;
     p.rb4 = kWarps * tl.rpw4;
     p.nrb4 = (c->d + p.rb4 - 1) / p.rb4;
+    if (tc) {  // tasks of up to kTcNT tokens; units of 128 gate/up rows, 256 down rows
+        p.tc = 1;
+        p.CH = kTcNT;
+        p.rb3 = 128;
+        p.nrb3 = (c->f + 127) / 128;
+        p.rb4 = 256;
+        p.nrb4 = (c->d + 255) / 256;
+    }
     p.ksplit = 1;
     const Dims l = layout_dims(c, ws_bytes);
     p.ws = ws_carve(l, ws);
@@ -177,7 +197,7 @@ static moe_status check_ws(const moe_config* c, int T, void* ws, size_t ws_bytes
 template <int TM, typename XT>
 static cudaError_t route_small_nv(Params& p, const XT* x, int do_quant, int bucket, cudaStream_t s) {
     const int E = p.m.E;
-    const size_t smem = std::max((size_t)2 * kWarps * E * 4, (size_t)(4 * E + kWarps) * 4);
+    const size_t smem = std::max((size_t)2 * kWarps * E * 4, (size_t)(5 * E + kWarps) * 4);
     const int nv = p.m.d / 4;
     const int per = (nv + kThreads - 1) / kThreads;
     const int grid = (E + 1) / 2;
@@ -226,7 +246,7 @@ static cudaError_t launch_router(Params& p, const XT* x, int do_quant, int bucke
     k_topk<<<(T + kWarps - 1) / kWarps, kThreads, smem_topk, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (bucket) {
-        k_bucket<<<1, kThreads, (size_t)(4 * E + kWarps) * 4, s>>>(p);
+        k_bucket<<<1, kThreads, (size_t)(5 * E + kWarps) * 4, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -342,7 +362,13 @@ moe_status moe_expert_ffn(const moe_config* cfg, const moe_pool* pool, int32_t e
     MOE_TRY(check_ptr(dbg_sh, "dbg_sh", true));
     MOE_TRY(check_ptr(dbg_acc_d, "dbg_acc_d", true));
     const bool dbg = dbg_acc_gu || dbg_hq || dbg_sh || dbg_acc_d;
-    if (dbg) p.CH = 8;
+    const bool tc = use_tc(cfg, T);
+    if (tc) p = base_params(cfg, p.m, ws, ws_bytes, true);
+    else if (dbg) p.CH = 8;
+    p.pool = pool->w;
+    p.scales = pool->s;
+    p.direct_out = 1;
+    p.out = y;
     p.dbg_acc_gu = dbg_acc_gu;
     p.dbg_hq = dbg_hq;
     p.dbg_sh = dbg_sh;
@@ -355,8 +381,15 @@ moe_status moe_expert_ffn(const moe_config* cfg, const moe_pool* pool, int32_t e
     if (e != cudaSuccess) return cuda_fail(e, "moe_expert_ffn copy");
     k_sum_codes<<<std::min((int)T, 65535), kThreads, 0, s>>>(p.ws.xq, T, cfg->d, p.ws.xcs);
     k_plan_single<<<1, kThreads, 0, s>>>(p, blob);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "moe_expert_ffn");
+    if (tc) {
+        e = launch_tc_gather(p, p.ws.xq, cfg->d, 1, cfg->d, p.ws.xb, s);
+        if (e == cudaSuccess) e = launch_tc_expert(p, 0, tc_nt_max(T), s);
+        if (e == cudaSuccess) e = launch_tc_expert(p, 1, tc_nt_max(T), s);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn (tensor cores)");
+    }
     const ExpertTiling tl = expert_tiling(cfg->d, cfg->f, cfg->wbits);
-    if ((e = cudaGetLastError()) == cudaSuccess) e = launch_gate_up(p, tl, dbg, s);
+    e = launch_gate_up(p, tl, dbg, s);
     if (e == cudaSuccess) e = launch_down(p, tl, dbg, s);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn");
 }
@@ -371,13 +404,28 @@ moe_status moe_expert_down(const moe_config* cfg, const moe_pool* pool, int32_t 
     MOE_TRY(check_ptr(sh, "sh"));
     MOE_TRY(check_ptr(dbg_acc_d, "dbg_acc_d", true));
     const bool dbg = dbg_acc_d != nullptr;
-    if (dbg) p.CH = 8;
+    const bool tc = use_tc(cfg, T);
+    if (tc) p = base_params(cfg, p.m, ws, ws_bytes, true);
+    else if (dbg) p.CH = 8;
+    p.pool = pool->w;
+    p.scales = pool->s;
+    p.direct_out = 1;
+    p.out = y;
     p.hq_in = hq;
     p.sh_in = sh;
     p.dbg_acc_d = dbg_acc_d;
     cudaStream_t s = (cudaStream_t)stream;
     k_plan_single<<<1, kThreads, 0, s>>>(p, expert < 0 ? cfg->n_experts : expert);
     cudaError_t e = cudaGetLastError();
+    if (tc) {
+        if (e == cudaSuccess) {
+            k_sum_codes<<<std::min((int)T, 65535), kThreads, 0, s>>>(hq, T, cfg->f, p.ws.hcs);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = launch_tc_gather(p, hq, cfg->f, 1, cfg->f, p.ws.hb, s);
+        if (e == cudaSuccess) e = launch_tc_expert(p, 1, tc_nt_max(T), s);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_down (tensor cores)");
+    }
     if (e == cudaSuccess) e = launch_down(p, expert_tiling(cfg->d, cfg->f, cfg->wbits), dbg, s);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_down");
 }
@@ -390,7 +438,10 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     MOE_TRY(check_dtype(dtype));
     if (!pool) return fail(MOE_EINVAL, "pool is NULL");
     if (T < 0) return fail(MOE_EINVAL, "T < 0");
-    if (opts) opts->n_launches = 0;
+    if (opts) {
+        opts->n_launches = 0;
+        opts->path_ran = MOE_PATH_AUTO;
+    }
     if (T == 0) return MOE_OK;
     MOE_TRY(check_ptr(pool->w, "pool->w"));
     MOE_TRY(check_ptr(pool->s, "pool->s"));
@@ -419,17 +470,45 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         return cudaSuccess;
     };
     const int path = opts ? opts->path : MOE_PATH_AUTO;
-    if (path != MOE_PATH_AUTO && path != MOE_PATH_MULTI && path != MOE_PATH_DECODE)
-        return fail(MOE_EINVAL, "opts->path must be MOE_PATH_AUTO, MOE_PATH_MULTI or MOE_PATH_DECODE");
+    if (path != MOE_PATH_AUTO && path != MOE_PATH_MULTI && path != MOE_PATH_DECODE && path != MOE_PATH_TC)
+        return fail(MOE_EINVAL, "opts->path must be MOE_PATH_AUTO, MOE_PATH_MULTI, MOE_PATH_DECODE or MOE_PATH_TC");
     DecPlan pl{};
-    const bool dec_ok = path != MOE_PATH_MULTI && decode_plan(m, &pl);
+    const bool dec_ok = (path == MOE_PATH_AUTO || path == MOE_PATH_DECODE) && decode_plan(m, &pl);
     if (path == MOE_PATH_DECODE && !dec_ok) return fail(MOE_EINVAL, "shape does not fit the single-launch decode path");
+    if (path == MOE_PATH_TC && !tc_shape_ok(m)) return fail(MOE_EINVAL, "shape does not fit the tensor-core path");
     cudaError_t e = mark(0);
     if (dec_ok) {
         if (e == cudaSuccess) e = launch_decode(p, pl, x, dtype == MOE_BF16, s);
         for (int i = 1; i < 4 && e == cudaSuccess; ++i) e = mark(i);
-        if (opts) opts->n_launches = 1;
+        if (opts) {
+            opts->n_launches = 1;
+            opts->path_ran = MOE_PATH_DECODE;
+        }
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (decode)");
+    }
+    if (path == MOE_PATH_TC || (path == MOE_PATH_AUTO && use_tc(cfg, T))) {
+        Params q = base_params(cfg, m, ws, ws_bytes, true);
+        q.pool = p.pool;
+        q.scales = p.scales;
+        q.w_router = p.w_router;
+        q.bias = p.bias;
+        q.out = p.out;
+        q.accumulate = p.accumulate;
+        q.idx_out = p.idx_out;
+        q.w_out = p.w_out;
+        if (e == cudaSuccess) e = launch_router_any(q, x, dtype, 1, 1, s);
+        if (e == cudaSuccess) e = launch_tc_gather(q, q.ws.xq, cfg->d, m.S, cfg->d, q.ws.xb, s);
+        if (e == cudaSuccess) e = mark(1);
+        if (e == cudaSuccess) e = launch_tc_expert(q, 0, tc_nt_max(T), s);
+        if (e == cudaSuccess) e = mark(2);
+        if (e == cudaSuccess) e = launch_tc_expert(q, 1, tc_nt_max(T), s);
+        if (e == cudaSuccess) e = launch_combine(q, s);
+        if (e == cudaSuccess) e = mark(3);
+        if (opts) {
+            opts->n_launches = (T <= 8 ? 1 : 4) + 4;
+            opts->path_ran = MOE_PATH_TC;
+        }
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (tensor cores)");
     }
     if (e == cudaSuccess) e = launch_router_any(p, x, dtype, 1, 1, s);
     if (e == cudaSuccess) e = mark(1);
@@ -437,7 +516,10 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     if (e == cudaSuccess) e = mark(2);
     if (e == cudaSuccess) e = launch_down(p, tl, false, s);
     if (e == cudaSuccess) e = mark(3);
-    if (opts) opts->n_launches = (T <= 8 ? 1 : 4) + 2;
+    if (opts) {
+        opts->n_launches = (T <= 8 ? 1 : 4) + 2;
+        opts->path_ran = MOE_PATH_MULTI;
+    }
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer");
 }
 

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "moe.h"
 
 namespace moe {
@@ -57,6 +59,9 @@ struct Ws {
     float* sh;         // [T*S]      scale of hq
     float* ybuf;       // [T*S][d]   per-assignment down outputs before the combine
     uint32_t* rb_ctr;  // [ceil(d/rb4)] down item arrivals per row block (self-resetting)
+    int32_t* hcs;      // [T*S]      sum of the hq codes of each assignment (tensor-core down)
+    uint8_t* xb;       // tensor-core operand B of gate/up: per task, activation rows in MMA layout
+    uint8_t* hb;       // tensor-core operand B of down: per task, hq rows in MMA layout
     size_t bytes;
 };
 
@@ -69,6 +74,20 @@ struct Dims {
 };
 
 inline int max_tasks(const Dims& m) { return m.T * m.S + m.E + 2; }
+
+// Tensor-core path: tasks hold at most kTcNT tokens (the MMA N), padded to
+// tc_npad rows; a K chunk is 64 packed weight bytes (128 int4 / 256 int2 codes).
+constexpr int kTcNT = 128;
+__host__ __device__ constexpr int tc_npad(int n) { return n <= 8 ? 8 : (n + 15) & ~15; }
+__host__ __device__ constexpr int tc_kc(int wb) { return 512 / wb; }
+__host__ __device__ constexpr int tc_kpad(int k, int wb) { return (k + tc_kc(wb) - 1) / tc_kc(wb) * tc_kc(wb); }
+// Bound on the padded rows of all tasks of a call: every task has >= 1 token
+// and pads by < 16 rows; tasks <= experts present + assignments / kTcNT.
+inline size_t tc_rows_bound(const Dims& m) {
+    const size_t A = (size_t)m.T * m.S;
+    const size_t tasks = std::min(A, (size_t)(m.E + m.has_shared) + (A + kTcNT - 1) / kTcNT);
+    return A + 15 * tasks;
+}
 // Rows per warp per work item of the gate/up and down kernels (one definition
 // for the kernels' template arguments and the host's item counts).
 constexpr int rpw3() { return 2; }
@@ -103,6 +122,9 @@ inline Ws ws_carve(const Dims& m, void* base) {
     w.sh = (float*)take(A * 4);
     w.ybuf = (float*)take(A * m.d * 4);
     w.rb_ctr = (uint32_t*)take((size_t)((m.d + kMinRowBlock4 - 1) / kMinRowBlock4) * 4);
+    w.hcs = (int32_t*)take(A * 4);
+    w.xb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.d, m.wb));
+    w.hb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.f, m.wb));
     w.bytes = off;
     return w;
 }
@@ -134,6 +156,7 @@ struct Params {
     int rb3, nrb3;   // gate/up rows per item, items per task
     int rb4, nrb4;   // down rows per item, items per task
     int ksplit;      // router split of d
+    int tc;          // tasks are tensor-core tasks (<= kTcNT tokens, padded-row offsets in task.w)
     Ws ws;
     int a_cap;       // assignments the workspace layout holds (capacity T x S)
     unsigned long long* trace;  // optional per-CTA phase stamps of the decode kernel
@@ -241,6 +264,105 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
 }
 __device__ __forceinline__ int ld_volatile_status(const WsHeader* h) {
     return *reinterpret_cast<const volatile int*>(&h->status);
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core (tcgen05) and 2-D TMA wrappers (sm_100a)
+// ---------------------------------------------------------------------------
+// 2-D tiled TMA load of box {x bytes, y rows} at coordinates (x, y) into this
+// CTA's shared memory; completion counted in bytes on `bar`.  No multicast.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// TMEM allocation by one full warp; the column base is written to *dst_smem.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Shared-memory matrix descriptor, no swizzle, K-major core matrices of 8 rows
+// x 16 bytes: lbo = byte distance of K-adjacent core matrices, sbo = of
+// M/N-adjacent 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// D[tmem] (+)= A[tmem] x B[smem]^T, 8-bit x 8-bit -> int32, M = 128, one CTA.
+// A: row i in TMEM lane i, K bytes packed four to a 32-bit column.
+__device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p; }" ::"r"(
+            d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on `bar` once every tcgen05.mma this thread issued before has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, int v[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, int v[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 16 / 32 consecutive 32-bit TMEM columns of this thread's lane <- registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t v[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t v[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Instruction descriptor of tcgen05.mma.kind::i8: D s32, A unsigned 8-bit
+// (offset-binary weight codes), B signed 8-bit (activations), both K-major,
+// M = 128, N = 8 or a multiple of 16 up to 256.
+__host__ __device__ constexpr uint32_t tc_idesc_u8s8(int n) {
+    return (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+// L2 policy for data read exactly once (the weight stream).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
 }
 
 // Bound of every device-side wait: after this long the waiter records

@@ -1,0 +1,105 @@
+// Host side of the tensor-core expert path: tensor maps over the expert pool,
+// shared-memory plan, and the launches of the gather, gate/up, down and
+// combine kernels (moe_tc.cuh).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "moe_launch.h"
+#include "moe_tc.cuh"
+
+namespace moe {
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D uint8 view of the pool: `rows` rows of `rowbytes` bytes; box of
+// 64 bytes x 128 rows, 64-byte swizzle, zero fill outside the tensor.
+static cudaError_t make_pool_map(CUtensorMap* tm, const void* pool, uint64_t rowbytes, uint64_t rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {rowbytes, rows};
+    const cuuint64_t strides[1] = {rowbytes};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pool), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Largest shared-memory footprint a CTA may take, and the slot count that
+// fills it; always large enough that one CTA occupies an SM (TMEM is
+// allocated whole).
+constexpr size_t kTcSmemBudget = 227 * 1024;
+
+static int tc_slots(int nt_max, int wb) {
+    const size_t room = kTcSmemBudget - 1024 - sizeof(TcCtl);
+    return (int)std::min<size_t>(kTcMaxSlots, room / tc_slot_bytes(nt_max, wb));
+}
+
+bool tc_shape_ok(const Dims& m) {
+    // every assignment's token count fits the task split, and the slot ring
+    // holds at least two chunks
+    return tc_slots(kTcNT, m.wb) >= 2 && m.d <= 8192 && m.f <= 8192;
+}
+
+template <int WB, int EPI>
+static cudaError_t launch_tc_t(const Params& p, const CUtensorMap& tm, int nt_max, cudaStream_t s) {
+    const int ns = tc_slots(nt_max, WB);
+    const size_t smem = std::max(tc_smem_bytes(ns, nt_max, WB), (size_t)120 * 1024);
+    auto fn = k_tc<WB, EPI>;
+    cudaError_t e = allow_smem((const void*)fn, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    fn<<<sms, kTcThreads, smem, s>>>(p, tm, ns, nt_max);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_t s) {
+    const int E1 = p.m.E + p.m.has_shared;
+    CUtensorMap tm;
+    const int wb = p.m.wb;
+    cudaError_t e;
+    if (stage == 0)
+        e = make_pool_map(&tm, p.pool, (uint64_t)p.m.d * wb / 8, (uint64_t)3 * p.m.f * E1);
+    else
+        e = make_pool_map(&tm, p.pool, (uint64_t)p.m.f * wb / 8, (uint64_t)3 * p.m.d * E1);
+    if (e != cudaSuccess) return e;
+    if (wb == 4) return stage == 0 ? launch_tc_t<4, 0>(p, tm, nt_max, s) : launch_tc_t<4, 1>(p, tm, nt_max, s);
+    return stage == 0 ? launch_tc_t<2, 0>(p, tm, nt_max, s) : launch_tc_t<2, 1>(p, tm, nt_max, s);
+}
+
+cudaError_t launch_tc_gather(const Params& p, const int8_t* src, int ld, int key_div, int K, uint8_t* dst,
+                             cudaStream_t s) {
+    const int kpad = tc_kpad(K, p.m.wb);
+    const int grid = 2 * persistent_grid((const void*)k_tc_gather<4>, 0);
+    if (p.m.wb == 4) k_tc_gather<4><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
+    else k_tc_gather<2><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Params& p, cudaStream_t s) {
+    const size_t n4 = (size_t)p.m.T * (p.m.d / 4);
+    const int grid = (int)std::max<size_t>(1, std::min<size_t>((n4 + kThreads - 1) / kThreads,
+                                                               (size_t)persistent_grid((const void*)k_combine, 0)));
+    k_combine<<<grid, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -39,4 +39,15 @@ moe_status check_ptr(const void* p, const char* name, bool nullable = false);
 moe_status check_dtype(moe_dtype dt);
 cudaError_t launch_down(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s);
 
+// Tensor-core expert path (moe_ktc.cu).  nt_max: bound on the tokens of one
+// task in this call (<= kTcNT).
+bool tc_shape_ok(const Dims& m);
+// stage 0: gate/up (+ requantisation into the down operand), 1: down.
+cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_t s);
+// Operand B of every task from int8 rows `src` (row = assignment id / key_div).
+cudaError_t launch_tc_gather(const Params& p, const int8_t* src, int ld, int key_div, int K, uint8_t* dst,
+                             cudaStream_t s);
+// out (+)= weighted sum of the per-assignment down outputs, over the grid.
+cudaError_t launch_combine(const Params& p, cudaStream_t s);
+
 }  // namespace moe

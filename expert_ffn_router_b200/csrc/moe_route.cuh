@@ -119,8 +119,10 @@ static __device__ void topk_token(const Params& p, int t, float* s_sm, float* se
 // a2 by one CTA: group the T*k (token, slot) assignments by expert, stable in
 // (token, slot) order, append the shared expert's T assignments first, cut
 // each expert's list into tasks of at most CH tokens, publish the work-item
-// counts and zero the per-call counters of the expert kernels.
-// smem: 4 * E ints + kWarps ints.
+// counts and zero the per-call counters of the expert kernels.  For
+// tensor-core tasks (p.tc) task.w is the task's first row in the padded
+// operand buffers (the sum of tc_npad over the tasks before it).
+// smem: 5 * E ints + kWarps ints.
 static __device__ void bucket_cta(const Params& p, int* smem) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = p.m.E, k = p.m.k, T = p.m.T, S = p.m.S, CH = p.CH;
@@ -129,7 +131,8 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     int* off = smem + E;
     int* tb = smem + 2 * E;
     int* off0 = smem + 3 * E;
-    int* red = smem + 4 * E;
+    int* prow = smem + 4 * E;
+    int* red = smem + 5 * E;
     WsHeader* hdr = p.ws.hdr;
     for (int e = tid; e < E; e += kThreads) cnt[e] = 0;
     __syncthreads();
@@ -145,14 +148,17 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     for (int e = tid; e < E; e += kThreads) {
         off[e] = cnt[e];
         tb[e] = (cnt[e] + CH - 1) / CH;
+        prow[e] = (cnt[e] / CH) * tc_npad(CH) + (cnt[e] % CH ? tc_npad(cnt[e] % CH) : 0);
     }
     __syncthreads();
     block_exscan(off, E, red);
     const int n_routed_tasks = block_exscan(tb, E, red);
+    if (p.tc) block_exscan(prow, E, red);
     for (int e = tid; e < E; e += kThreads) off0[e] = off[e];
     __syncthreads();
     const int asg_base = p.m.has_shared ? T : 0;
     const int n_sh_tasks = p.m.has_shared ? (T + CH - 1) / CH : 0;
+    const int sh_rows = p.m.has_shared ? (T / CH) * tc_npad(CH) + (T % CH ? tc_npad(T % CH) : 0) : 0;
     if (warp == 0) {
         for (int base = 0; base < A; base += 32) {
             const int a = base + lane;
@@ -169,11 +175,12 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     if (p.m.has_shared)
         for (int t = tid; t < T; t += kThreads) p.ws.asg[t] = t * S + k;
     for (int c = tid; c < n_sh_tasks; c += kThreads)
-        p.ws.tasks[c] = make_int4(E, c * CH, min(CH, T - c * CH), 0);
+        p.ws.tasks[c] = make_int4(E, c * CH, min(CH, T - c * CH), p.tc ? c * tc_npad(CH) : 0);
     for (int e = tid; e < E; e += kThreads) {
         const int n = cnt[e];
         for (int c = 0; c * CH < n; ++c)
-            p.ws.tasks[n_sh_tasks + tb[e] + c] = make_int4(e, asg_base + off0[e] + c * CH, min(CH, n - c * CH), 0);
+            p.ws.tasks[n_sh_tasks + tb[e] + c] = make_int4(e, asg_base + off0[e] + c * CH, min(CH, n - c * CH),
+                                                           p.tc ? sh_rows + prow[e] + c * tc_npad(CH) : 0);
     }
     const int n_tasks = n_sh_tasks + n_routed_tasks;
     for (int i = tid; i < n_tasks; i += kThreads) p.ws.task_ctr[i] = 0;
@@ -191,7 +198,7 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
 // 2b+1 for every token (each thread a slice of d, weights streamed once); CTAs
 // b < T also quantise token b.  The last CTA to finish runs the top-k of every
 // token (one warp per token) and, if `bucket`, the bucketing.
-// Dynamic smem: max(2 * kWarps * E floats, 4 * E + kWarps ints).
+// Dynamic smem: max(2 * kWarps * E floats, 5 * E + kWarps ints).
 template <int TM, int NV, typename XT>
 __global__ void __launch_bounds__(kThreads) k_route_small(const Params p, const XT* __restrict__ x,
                                                           int do_quant, int bucket) {
@@ -338,7 +345,7 @@ __global__ void __launch_bounds__(kThreads) k_topk(const Params p) {
     if (t < p.m.T) topk_token(p, t, dsm + warp * 2 * p.m.E, dsm + warp * 2 * p.m.E + p.m.E);
 }
 
-// Bucketing alone (one CTA).  Dynamic smem (4 * E + kWarps) ints.
+// Bucketing alone (one CTA).  Dynamic smem (5 * E + kWarps) ints.
 __global__ void __launch_bounds__(kThreads) k_bucket(const Params p) {
     extern __shared__ int ism[];
     bucket_cta(p, ism);
@@ -354,7 +361,7 @@ __global__ void __launch_bounds__(kThreads) k_plan_single(const Params p, int bl
         p.ws.amax[t] = 0u;
     }
     for (int c = threadIdx.x; c < n_tasks; c += kThreads) {
-        p.ws.tasks[c] = make_int4(blob, c * CH, min(CH, T - c * CH), 0);
+        p.ws.tasks[c] = make_int4(blob, c * CH, min(CH, T - c * CH), p.tc ? c * tc_npad(CH) : 0);
         p.ws.task_ctr[c] = 0u;
     }
     for (int i = threadIdx.x; i < p.nrb4; i += kThreads) p.ws.rb_ctr[i] = 0u;

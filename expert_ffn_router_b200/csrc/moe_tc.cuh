@@ -1,0 +1,521 @@
+// Steps a3-a6 on the 5th-generation tensor cores (tcgen05, sm_100a): the
+// int8 grouped GEMM for batches whose experts see many tokens (prefill,
+// long verify batches).  An expert's packed weights stream from HBM once per
+// task of up to kTcNT tokens; the integer products run as
+// tcgen05.mma.kind::i8 with int32 accumulators in tensor memory (TMEM).
+//
+// Operands (one MMA: M = 128 weight rows, N = the task's padded tokens,
+// K = 32 codes):
+//  A  weight codes.  A TMA box of 128 rows x 64 packed bytes (64-byte swizzle)
+//     lands in shared memory; the unpack warps split each 32-bit word into
+//     offset-binary bytes (u = c + 8 for int4, c + 2 for int2, the same masks
+//     as the dp4a kernels) and store them to TMEM, from where the MMA reads A.
+//     Unsigned A times signed activations gives sum(u x) = sum(c x) + off sum(x);
+//     the epilogue subtracts off * sum(x).
+//  B  int8 activations (or requantised h) of the task's tokens, in the
+//     canonical K-major no-swizzle layout of 8-row x 16-byte core matrices,
+//     with each 16-byte K group in the byte order the unpack produces
+//     (permute16).  A gather kernel (x) or the gate/up epilogue (h) writes it
+//     per task and K chunk, so one bulk copy brings a chunk's B into shared
+//     memory.
+//
+// Persistent kernel, one CTA per SM, 320 threads:
+//  warp 0    TMA producer: per K chunk two A boxes + the B chunk into a ring
+//            of shared-memory slots (full / empty mbarriers);
+//  warp 1    TMEM allocator and MMA issuer (one thread): per chunk
+//            KC/32 K-steps x 2 tiles, tcgen05.commit releases the slot and the
+//            TMEM A buffer, a final commit per unit hands the accumulators to
+//            the epilogue;
+//  warps 2-9 unpack A into one of two TMEM A buffers, then run the epilogue
+//            (tcgen05.ld of the accumulators).
+// A unit is (task, row block): two 128-row A tiles sharing one B --
+//  gate/up (EPI 0): gate rows and up rows [128 rb, 128 rb + 128) of f;
+//                   epilogue h = SiLU(g) u, per-token max |h|; the CTA that
+//                   completes a task's last unit requantises the task's h
+//                   into the down operand (hb), its scales and code sums.
+//  down    (EPI 1): rows [256 rb, 256 rb + 256) of d as two tiles; epilogue
+//                   y = acc (s_row s_h) to the per-assignment buffer (the
+//                   combine is a separate kernel) or straight to the output.
+// TMEM columns: [0, 128) tile-0 accumulators, [128, 256) tile 1, then two A
+// buffers of 2 x KC/4 columns.  Every wait is bounded (kWaitLimitNs); on a
+// timeout the CTA records MOE_ETIMEOUT, lets its copies and MMAs drain and
+// exits.
+#pragma once
+
+#include <cuda.h>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kTcThreads = 320;
+constexpr int kTcEpi = 256;                    // unpack / epilogue threads (warps 2-9)
+constexpr int kTcBox = 128 * 64;               // one A box: 128 rows x 64 packed bytes
+constexpr int kTcSlotA = 2 * kTcBox;           // both tiles of a chunk
+constexpr int kTcMaxSlots = 8;
+
+// Dynamic shared memory: [slots][control block], slots 1024-byte aligned.
+struct TcCtl {
+    uint64_t full[kTcMaxSlots], empty[kTcMaxSlots];
+    uint64_t afull[2], afree[2], accfull, accempty, drain;
+    uint32_t tmem_base;
+    int last;
+    int asg[2][kTcNT];
+    float sx[2][kTcNT];
+    int cs[2][kTcNT];
+    unsigned amax[kTcNT];
+    int hcs[kTcNT];
+};
+
+__host__ __device__ constexpr int tc_slot_bytes(int nt_max, int wb) {
+    return (kTcSlotA + nt_max * tc_kc(wb) + 1023) / 1024 * 1024;
+}
+__host__ __device__ constexpr size_t tc_smem_bytes(int ns, int nt_max, int wb) {
+    return 1024 + (size_t)ns * tc_slot_bytes(nt_max, wb) + sizeof(TcCtl);
+}
+
+// Same as mbar_wait_bounded, but also gives up when another wait of the call
+// has already failed (the status word is set).
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 255u) {
+            if (ld_volatile_status(hdr) != 0) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                set_status(hdr, MOE_ETIMEOUT, site);
+                return false;
+            }
+        }
+    }
+}
+
+// Unpack one thread's share of one A tile of a chunk into TMEM.  Row `row` of
+// the box (64 packed bytes, 64-byte swizzle: 16-byte unit j of row r sits at
+// unit j ^ ((r >> 1) & 3)); half `hh` takes units 2hh and 2hh+1.
+template <int WB>
+__device__ __forceinline__ void tc_unpack_tile(const uint8_t* box, int row, int hh, uint32_t taddr) {
+    const uint8_t* rp = box + row * 64;
+    const int sw = (row >> 1) & 3;
+    if (WB == 4) {
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + (((2 * hh + j) ^ sw) << 4));
+            const uint32_t in[4] = {v.x ^ 0x88888888u, v.y ^ 0x88888888u, v.z ^ 0x88888888u, v.w ^ 0x88888888u};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                w[8 * j + 2 * i] = in[i] & 0x0F0F0F0Fu;
+                w[8 * j + 2 * i + 1] = (in[i] >> 4) & 0x0F0F0F0Fu;
+            }
+        }
+        tmem_st16(taddr, w);
+    } else {
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + (((2 * hh + j) ^ sw) << 4));
+            const uint32_t in[4] = {v.x ^ 0xAAAAAAAAu, v.y ^ 0xAAAAAAAAu, v.z ^ 0xAAAAAAAAu, v.w ^ 0xAAAAAAAAu};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int s = 0; s < 4; ++s) w[16 * j + 4 * i + s] = (in[i] >> (2 * s)) & 0x03030303u;
+        }
+        tmem_st32(taddr, w);
+    }
+}
+
+// Byte offset of 16-byte K group `kg` (K columns 16 kg .. 16 kg + 15) of
+// padded row j in a task's B buffer, laid out [K group][row][16 bytes]: K
+// chunk c (KC columns) is the npad * KC bytes at c * npad * KC, and within it
+// the core matrix of rows 8i..8i+7 and K group g sits at (g * npad + 8i) * 16.
+__device__ __forceinline__ size_t tc_b_offset(int kg, int j, int npad) {
+    return ((size_t)kg * npad + j) * 16;
+}
+
+template <int WB, int EPI>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_tc(const Params p, const __grid_constant__ CUtensorMap tmA, int ns, int nt_max) {
+    constexpr int KC = tc_kc(WB);         // K columns per chunk
+    constexpr int ACOLS = KC / 4;         // TMEM columns of one tile's A chunk
+    constexpr int KSTEPS = KC / 32;
+    constexpr int OFF = code_offset<WB>();
+    extern __shared__ uint8_t tc_raw[];
+    uint8_t* base = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023u)) & 1023u);
+    const int slot_bytes = tc_slot_bytes(nt_max, WB);
+    TcCtl* ctl = reinterpret_cast<TcCtl*>(base + (size_t)ns * slot_bytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    WsHeader* hdr = p.ws.hdr;
+    const int d = p.m.d, f = p.m.f;
+    const int K = EPI == 0 ? d : f;
+    const int nch = (K + KC - 1) / KC;
+    const int kpad = nch * KC;
+    const int nrb = EPI == 0 ? (f + 127) / 128 : (d + 255) / 256;
+    const int n_units = hdr->n_tasks * nrb;
+    const uint8_t* bbuf = EPI == 0 ? p.ws.xb : p.ws.hb;
+
+    if (tid == 0) {
+        for (int i = 0; i < ns; ++i) {
+            mbar_init(&ctl->full[i], 1);
+            mbar_init(&ctl->empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->afull[i], kTcEpi);
+            mbar_init(&ctl->afree[i], 1);
+        }
+        mbar_init(&ctl->accfull, 1);
+        mbar_init(&ctl->accempty, kTcEpi);
+        mbar_init(&ctl->drain, 1);
+        fence_mbar_init();
+    }
+    if (tid >= 64) {
+        ctl->amax[(tid - 64) & (kTcNT - 1)] = 0u;
+        ctl->hcs[(tid - 64) & (kTcNT - 1)] = 0;
+    }
+    if (warp == 1) tmem_alloc(&ctl->tmem_base, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = ctl->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            int slot = 0;
+            uint32_t ph = 0, issued = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const int ti = u / nrb, rb = u - ti * nrb;
+                const int4 task = p.ws.tasks[ti];
+                const int npad = tc_npad(task.z);
+                const uint32_t bbytes = (uint32_t)npad * KC;
+                int y0, y1;
+                if (EPI == 0) {
+                    y0 = task.x * 3 * f + rb * 128;
+                    y1 = y0 + f;
+                } else {
+                    y0 = task.x * 3 * d + 2 * d + rb * 256;
+                    y1 = y0 + 128;
+                }
+                const uint8_t* bsrc = bbuf + (size_t)task.w * kpad;
+                for (int c = 0; c < nch; ++c) {
+                    if (!tc_wait(&ctl->empty[slot], ph ^ 1u, hdr, 0x7101)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sp = base + (size_t)slot * slot_bytes;
+                    mbar_arrive_expect_tx(&ctl->full[slot], kTcSlotA + bbytes);
+                    tma_load_2d(sp, &tmA, c * 64, y0, &ctl->full[slot], pol);
+                    tma_load_2d(sp + kTcBox, &tmA, c * 64, y1, &ctl->full[slot], pol);
+                    bulk_g2s(sp + kTcSlotA, bsrc + (size_t)c * bbytes, bbytes, &ctl->full[slot]);
+                    ++issued;
+                    if (++slot == ns) {
+                        slot = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // drain: every issued copy has landed before the CTA exits
+            for (int s = 0; s < ns; ++s) {
+                const uint32_t n_s = issued / ns + ((uint32_t)s < issued % ns ? 1u : 0u);
+                if (n_s) mbar_wait_bounded(&ctl->full[s], (n_s - 1) & 1u, hdr, 0x7102);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int slot = 0;
+            uint32_t ph = 0, g = 0, uidx = 0;
+            bool ok = true, issued = false;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++uidx) {
+                const int ti = u / nrb;
+                const int npad = tc_npad(p.ws.tasks[ti].z);
+                const uint32_t idesc = tc_idesc_u8s8(npad);
+                const uint32_t lbo = (uint32_t)npad * 16;
+                if (!tc_wait(&ctl->accempty, (uidx & 1u) ^ 1u, hdr, 0x7103)) break;
+                tc_fence_after();
+                for (int c = 0; c < nch; ++c, ++g) {
+                    const uint32_t ab = g & 1u;
+                    if (!tc_wait(&ctl->full[slot], ph, hdr, 0x7104) ||
+                        !tc_wait(&ctl->afull[ab], (g >> 1) & 1u, hdr, 0x7105)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t bsm = smem_u32(base + (size_t)slot * slot_bytes + kTcSlotA);
+                    const uint32_t acol = tbase + 256 + ab * 2 * ACOLS;
+#pragma unroll
+                    for (int ks = 0; ks < KSTEPS; ++ks) {
+                        const uint64_t bdesc = smem_desc(bsm + ks * 2 * lbo, lbo, 128);
+                        const uint32_t acc = (c | ks) != 0;
+                        tc_mma_i8_ts(tbase, acol + ks * 8, bdesc, idesc, acc);
+                        tc_mma_i8_ts(tbase + 128, acol + ACOLS + ks * 8, bdesc, idesc, acc);
+                    }
+                    issued = true;
+                    tc_commit(&ctl->empty[slot]);
+                    tc_commit(&ctl->afree[ab]);
+                    if (++slot == ns) {
+                        slot = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (ok) tc_commit(&ctl->accfull);
+            }
+            // drain: every MMA issued has completed before TMEM is released
+            if (issued) {
+                tc_commit(&ctl->drain);
+                mbar_wait_bounded(&ctl->drain, 0, hdr, 0x7106);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ unpack + epilogue
+        const int etid = tid - 64;
+        const int ew = warp - 2;
+        const int q = warp & 3;            // TMEM lane quarter this warp may access
+        const int hh = ew >> 2;            // which half of a chunk's units / of the tokens
+        const int row = 32 * q + lane;     // row of the 128-row tiles
+        const uint32_t tlane = tbase + ((uint32_t)(32 * q) << 16);
+        // A failed wait (timeout, or another wait of the call failed) makes
+        // `ok` false for the whole warp; the thread then skips the tensor-memory
+        // work but still arrives on every mbarrier and reaches every named
+        // barrier, so no thread of the CTA is left waiting.
+        int slot = 0;
+        uint32_t ph = 0, g = 0, uidx = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++uidx) {
+            const int ti = u / nrb, rb = u - ti * nrb;
+            const int4 task = p.ws.tasks[ti];
+            const int n = task.z, npad = tc_npad(n);
+            const int mb = uidx & 1;
+            if (etid < n) {
+                const int a = p.ws.asg[task.y + etid];
+                ctl->asg[mb][etid] = a;
+                if (EPI == 0) {
+                    const int tok = a / p.m.S;
+                    ctl->sx[mb][etid] = p.ws.sx[tok];
+                    ctl->cs[mb][etid] = p.ws.xcs[tok];
+                } else {
+                    ctl->sx[mb][etid] = p.sh_in ? p.sh_in[a] : __ldcg(p.ws.sh + a);
+                    ctl->cs[mb][etid] = __ldcg(p.ws.hcs + a);
+                }
+            }
+            for (int c = 0; c < nch; ++c, ++g) {
+                const uint32_t ab = g & 1u;
+                if (ok) ok = tc_wait(&ctl->full[slot], ph, hdr, 0x7107) &&
+                             tc_wait(&ctl->afree[ab], ((g >> 1) & 1u) ^ 1u, hdr, 0x7108);
+                ok = __all_sync(kFull, ok);
+                if (ok) {
+                    tc_fence_after();
+                    const uint8_t* sp = base + (size_t)slot * slot_bytes;
+                    const uint32_t acol = tlane + 256 + ab * 2 * ACOLS + hh * (ACOLS / 2);
+                    tc_unpack_tile<WB>(sp, row, hh, acol);
+                    tc_unpack_tile<WB>(sp + kTcBox, row, hh, acol + ACOLS);
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                mbar_arrive(&ctl->afull[ab]);
+                if (++slot == ns) {
+                    slot = 0;
+                    ph ^= 1u;
+                }
+            }
+            named_sync(1, kTcEpi);  // token metadata of this unit staged
+            if (ok) ok = tc_wait(&ctl->accfull, uidx & 1u, hdr, 0x7109);
+            ok = __all_sync(kFull, ok);
+            tc_fence_after();
+            if (ok && EPI == 0) {
+                const int r = rb * 128 + row;
+                const bool rv = r < f;
+                const float sg = rv ? __ldg(p.scales + (size_t)task.x * p.scale_rows + r) : 0.0f;
+                const float su = rv ? __ldg(p.scales + (size_t)task.x * p.scale_rows + f + r) : 0.0f;
+                for (int tg = hh; tg * 8 < npad; tg += 2) {
+                    int G[8], U[8];
+                    tmem_ld8(tlane + tg * 8, G);
+                    tmem_ld8(tlane + 128 + tg * 8, U);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int t = tg * 8 + j;
+                        if (t >= n) break;
+                        const int a = ctl->asg[mb][t];
+                        const float sx = ctl->sx[mb][t];
+                        const int gi = G[j] - OFF * ctl->cs[mb][t];
+                        const int ui = U[j] - OFF * ctl->cs[mb][t];
+                        const float gv = __fmul_rn((float)gi, __fmul_rn(sg, sx));
+                        const float uv = __fmul_rn((float)ui, __fmul_rn(su, sx));
+                        const float h = __fmul_rn(__fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv))), uv);
+                        if (rv) {
+                            p.ws.h[(size_t)a * f + r] = h;
+                            if (p.dbg_acc_gu) {
+                                p.dbg_acc_gu[(size_t)a * 2 * f + r] = gi;
+                                p.dbg_acc_gu[(size_t)a * 2 * f + f + r] = ui;
+                            }
+                        }
+                        const unsigned m = __reduce_max_sync(kFull, rv ? __float_as_uint(fabsf(h)) : 0u);
+                        if (lane == 0) atomicMax(&ctl->amax[t], m);
+                    }
+                }
+            } else if (ok) {
+                const int r0 = rb * 256 + row;
+                const float* sd = p.scales + (size_t)task.x * p.scale_rows + 2 * f;
+                const float s0 = r0 < d ? __ldg(sd + r0) : 0.0f;
+                const float s1 = r0 + 128 < d ? __ldg(sd + r0 + 128) : 0.0f;
+                float* dst = p.direct_out ? p.out : p.ws.ybuf;
+                for (int tg = hh; tg * 8 < npad; tg += 2) {
+                    int D0[8], D1[8];
+                    tmem_ld8(tlane + tg * 8, D0);
+                    tmem_ld8(tlane + 128 + tg * 8, D1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int t = tg * 8 + j;
+                        if (t >= n) break;
+                        const int a = ctl->asg[mb][t];
+                        const float sh = ctl->sx[mb][t];
+                        const int d0 = D0[j] - OFF * ctl->cs[mb][t];
+                        const int d1 = D1[j] - OFF * ctl->cs[mb][t];
+                        if (r0 < d) {
+                            dst[(size_t)a * d + r0] = __fmul_rn((float)d0, __fmul_rn(s0, sh));
+                            if (p.dbg_acc_d) p.dbg_acc_d[(size_t)a * d + r0] = d0;
+                        }
+                        if (r0 + 128 < d) {
+                            dst[(size_t)a * d + r0 + 128] = __fmul_rn((float)d1, __fmul_rn(s1, sh));
+                            if (p.dbg_acc_d) p.dbg_acc_d[(size_t)a * d + r0 + 128] = d1;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&ctl->accempty);
+            if (EPI == 0) {
+                named_sync(1, kTcEpi);  // per-token maxima of this CTA complete
+                if (etid < n) {
+                    atomicMax(&p.ws.amax[ctl->asg[mb][etid]], ctl->amax[etid]);
+                    ctl->amax[etid] = 0u;
+                }
+                __threadfence();        // this thread's h stores and maxima before the task count
+                named_sync(1, kTcEpi);
+                if (etid == 0) {
+                    __threadfence();
+                    ctl->last = ok && atomicAdd(&p.ws.task_ctr[ti], 1u) == (unsigned)(nrb - 1);
+                }
+                named_sync(1, kTcEpi);
+                if (ctl->last) {
+                    // every unit of this task is done: requantise its h (a4's
+                    // input rule) into the down operand, in the MMA layout
+                    __threadfence();
+                    if (etid == 0) p.ws.task_ctr[ti] = 0u;
+                    const int npk = tc_kpad(f, WB) / 16;  // 16-column groups per padded row
+                    uint8_t* hb = p.ws.hb + (size_t)task.w * tc_kpad(f, WB);
+                    for (int it = etid; it < npad * npk; it += kTcEpi) {
+                        const int j = it / npk, kg = it - j * npk;
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (j < n && kg * 16 < f) {
+                            const int a = ctl->asg[mb][j];
+                            const float m = __uint_as_float(__ldcg(p.ws.amax + a));
+                            if (m != 0.0f) {
+                                const float sh = __fdiv_rn(m, 127.0f);
+                                const float4* hp = reinterpret_cast<const float4*>(p.ws.h + (size_t)a * f + kg * 16);
+                                uint32_t wv[4];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const float4 hv = __ldcg(hp + i);
+                                    wv[i] = (uint32_t)(quant_code(hv.x, sh) & 0xFF) |
+                                            ((uint32_t)(quant_code(hv.y, sh) & 0xFF) << 8) |
+                                            ((uint32_t)(quant_code(hv.z, sh) & 0xFF) << 16) |
+                                            ((uint32_t)(quant_code(hv.w, sh) & 0xFF) << 24);
+                                }
+                                v = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                            }
+                            atomicAdd(&ctl->hcs[j], sum16(v));
+                            if (p.dbg_hq) *reinterpret_cast<uint4*>(p.dbg_hq + (size_t)a * f + kg * 16) = v;
+                        }
+                        *reinterpret_cast<uint4*>(hb + tc_b_offset(kg, j, npad)) = permute16<WB>(v);
+                    }
+                    named_sync(1, kTcEpi);  // every read of the task's maxima above is done
+                    if (etid < n) {
+                        const int a = ctl->asg[mb][etid];
+                        const float m = __uint_as_float(__ldcg(p.ws.amax + a));
+                        const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+                        p.ws.sh[a] = sh;
+                        p.ws.hcs[a] = ctl->hcs[etid];
+                        if (p.dbg_sh) p.dbg_sh[a] = sh;
+                        ctl->hcs[etid] = 0;
+                        p.ws.amax[a] = 0u;  // leave the workspace's maxima zeroed for the next call
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
+// Build the gate/up operand B of every task: the int8 rows of the task's
+// tokens (row key = assignment id / key_div of `src`, `ld` bytes apart),
+// K columns [0, K) zero-padded to kpad and rows padded to tc_npad, in the
+// MMA layout with permute16 byte order.
+template <int WB>
+__global__ void __launch_bounds__(kThreads) k_tc_gather(const Params p, const int8_t* __restrict__ src, int ld,
+                                                        int key_div, int K, int kpad, uint8_t* __restrict__ dst) {
+    const int n_tasks = p.ws.hdr->n_tasks;
+    const int npk = kpad / 16;
+    for (int ti = blockIdx.x; ti < n_tasks; ti += gridDim.x) {
+        const int4 task = p.ws.tasks[ti];
+        const int n = task.z, npad = tc_npad(n);
+        uint8_t* out = dst + (size_t)task.w * kpad;
+        for (int it = threadIdx.x; it < npad * npk; it += kThreads) {
+            const int j = it / npk, kg = it - j * npk;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (j < n && kg * 16 < K) {
+                const int key = p.ws.asg[task.y + j] / key_div;
+                v = __ldcg(reinterpret_cast<const uint4*>(src + (size_t)key * ld + kg * 16));
+            }
+            *reinterpret_cast<uint4*>(out + tc_b_offset(kg, j, npad)) = permute16<WB>(v);
+        }
+    }
+}
+
+// a6 over the whole grid: out[t] (+)= sum_j w_tj y_(t,j) + y_(t,shared),
+// summed in slot order (the same order as the row-block combine of k_down).
+__global__ void __launch_bounds__(kThreads) k_combine(const Params p) {
+    const int d = p.m.d, S = p.m.S, k = p.m.k, T = p.m.T;
+    const int nq = d / 4;
+    for (size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x; i < (size_t)T * nq; i += (size_t)gridDim.x * kThreads) {
+        const int t = (int)(i / nq), c4 = (int)(i - (size_t)t * nq) * 4;
+        float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int j = 0; j < k; ++j) {
+            const float w = __ldcg(p.ws.w + (size_t)t * k + j);
+            const float4 y = __ldcg(reinterpret_cast<const float4*>(p.ws.ybuf + ((size_t)t * S + j) * d + c4));
+            o.x = fmaf(w, y.x, o.x);
+            o.y = fmaf(w, y.y, o.y);
+            o.z = fmaf(w, y.z, o.z);
+            o.w = fmaf(w, y.w, o.w);
+        }
+        if (p.m.has_shared) {
+            const float4 y = __ldcg(reinterpret_cast<const float4*>(p.ws.ybuf + ((size_t)t * S + k) * d + c4));
+            o.x += y.x;
+            o.y += y.y;
+            o.z += y.z;
+            o.w += y.w;
+        }
+        float4* dp = reinterpret_cast<float4*>(p.out + (size_t)t * d + c4);
+        if (p.accumulate) {
+            const float4 b = *dp;
+            o.x += b.x;
+            o.y += b.y;
+            o.z += b.z;
+            o.w += b.w;
+        }
+        *dp = o;
+    }
+}
+
+}  // namespace moe

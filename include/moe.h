@@ -74,8 +74,10 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  *  top_k: experts per token k; has_shared: 1 if a shared expert follows the E
  *  routed blobs; wbits: 4 or 2; routed_scale: factor on the renormalised
  *  routed weights (2.5 for GLM-5.2).
- *  tc_min_tokens: experts with at least this many tokens in a call run on the
- *  int8 tensor-core (tcgen05) path; 0 = library default, < 0 = never.
+ *  tc_min_tokens: calls of at least this many tokens run the experts on the
+ *  int8 tensor-core (tcgen05) path (moe_layer with MOE_PATH_AUTO once the
+ *  single-launch decode path does not apply, moe_expert_ffn, moe_expert_down);
+ *  0 = library default (16), < 0 = never.
  * Limits (MOE_EINVAL otherwise): 1 <= k <= min(E, 32); E <= 1024;
  * d * wbits / 8 and f * wbits / 8 multiples of 16; d <= 8192; f <= 8192. */
 typedef struct {
@@ -170,8 +172,13 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *          The single-launch decode path records [0] before and [1..3] after
  *          its one kernel.
  *  path: MOE_PATH_AUTO (0), MOE_PATH_MULTI (1: separate routing, gate/up and
- *        down kernels) or MOE_PATH_DECODE (2: one persistent kernel for
- *        T <= 8; MOE_EINVAL if the shape does not fit it).
+ *        down kernels on dp4a integer dots), MOE_PATH_DECODE (2: one
+ *        persistent kernel for T <= 8; MOE_EINVAL if the shape does not fit
+ *        it) or MOE_PATH_TC (3: routing, then gate/up and down as int8
+ *        grouped GEMMs on the tensor cores, tasks of up to 128 tokens per
+ *        expert, then the combine).  AUTO takes DECODE where it fits, else TC
+ *        when T >= tc_min_tokens, else MULTI.
+ *  path_ran: set to the path that ran (MOE_PATH_DECODE, _MULTI or _TC).
  *  n_launches: set to the number of kernels the call launched.
  *  trace: optional DEVICE buffer of (number of SMs) x 16 uint64 that the
  *         single-launch decode path fills with per-CTA global-timer stamps
@@ -181,13 +188,14 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *         [7] first down staging ready, [8] down done; producer: [12] rows
  *         known before routing issued, [13] routing received, [14] all rows
  *         issued, [15] all copies landed.  Untouched entries are left as is. */
-enum { MOE_PATH_AUTO = 0, MOE_PATH_MULTI = 1, MOE_PATH_DECODE = 2 };
+enum { MOE_PATH_AUTO = 0, MOE_PATH_MULTI = 1, MOE_PATH_DECODE = 2, MOE_PATH_TC = 3 };
 typedef struct {
     void* events[4];
     int32_t path;
     int32_t n_launches;
     void* trace;
-    int32_t reserved[4];
+    int32_t path_ran;
+    int32_t reserved[3];
 } moe_layer_opts;
 
 /* moe_layer with options (opts may be NULL, then identical to moe_layer). */

@@ -159,7 +159,9 @@ def run_layer_gpu(wl, dl, x, accumulate_into=None, path="auto", ws=None):
                 topk_idx_out=idx, topk_w_out=w, opts=opts)
     assert_ok(ws)
     if path == "auto" and T <= 8:
-        assert opts.n_launches == 1  # the single-launch decode kernel ran
+        assert opts.n_launches == 1 and opts.path_ran == M.MOE_PATH_DECODE  # the single-launch kernel ran
+    if path == "multi":
+        assert opts.path_ran == M.MOE_PATH_MULTI
     return out, idx.cpu().numpy(), w.cpu().numpy()
 
 
