@@ -197,7 +197,7 @@ static moe_status check_ws(const moe_config* c, int T, void* ws, size_t ws_bytes
 template <int TM, typename XT>
 static cudaError_t route_small_nv(Params& p, const XT* x, int do_quant, int bucket, cudaStream_t s) {
     const int E = p.m.E;
-    const size_t smem = std::max((size_t)2 * kWarps * E * 4, (size_t)(5 * E + kWarps) * 4);
+    const size_t smem = std::max((size_t)2 * kWarps * E * 4, (size_t)(5 * E + kWarps + kBucketStage) * 4);
     const int nv = p.m.d / 4;
     const int per = (nv + kThreads - 1) / kThreads;
     const int grid = (E + 1) / 2;
@@ -246,7 +246,9 @@ static cudaError_t launch_router(Params& p, const XT* x, int do_quant, int bucke
     k_topk<<<(T + kWarps - 1) / kWarps, kThreads, smem_topk, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (bucket) {
-        k_bucket<<<1, kThreads, (size_t)(5 * E + kWarps) * 4, s>>>(p);
+        const size_t smem_b = (size_t)(5 * E + kWarps + kBucketStage) * 4;
+        if ((e = allow_smem((const void*)k_bucket, smem_b)) != cudaSuccess) return e;
+        k_bucket<<<1, kThreads, smem_b, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -385,6 +387,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const moe_pool* pool, int32_t e
     if (tc) {
         e = launch_tc_gather(p, p.ws.xq, cfg->d, 1, cfg->d, p.ws.xb, s);
         if (e == cudaSuccess) e = launch_tc_expert(p, 0, tc_nt_max(T), s);
+        if (e == cudaSuccess) e = launch_tc_requant(p, s);
         if (e == cudaSuccess) e = launch_tc_expert(p, 1, tc_nt_max(T), s);
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn (tensor cores)");
     }
@@ -500,12 +503,13 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         if (e == cudaSuccess) e = launch_tc_gather(q, q.ws.xq, cfg->d, m.S, cfg->d, q.ws.xb, s);
         if (e == cudaSuccess) e = mark(1);
         if (e == cudaSuccess) e = launch_tc_expert(q, 0, tc_nt_max(T), s);
+        if (e == cudaSuccess) e = launch_tc_requant(q, s);
         if (e == cudaSuccess) e = mark(2);
         if (e == cudaSuccess) e = launch_tc_expert(q, 1, tc_nt_max(T), s);
         if (e == cudaSuccess) e = launch_combine(q, s);
         if (e == cudaSuccess) e = mark(3);
         if (opts) {
-            opts->n_launches = (T <= 8 ? 1 : 4) + 4;
+            opts->n_launches = (T <= 8 ? 1 : 4) + 5;
             opts->path_ran = MOE_PATH_TC;
         }
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (tensor cores)");

@@ -33,7 +33,8 @@ struct WsHeader {
     uint32_t epoch;       // calls of the persistent decode kernel so far
     uint32_t b1_count;    // its grid barrier: arrivals (self-resetting)
     uint32_t b1_gen;      // its grid barrier: epoch of the last completion
-    int32_t pad[54];
+    int32_t tc_rows;      // padded rows of all tensor-core tasks of this call
+    int32_t pad[53];
 };
 static_assert(sizeof(WsHeader) == 256, "header must stay 256 bytes");
 
@@ -77,7 +78,7 @@ inline int max_tasks(const Dims& m) { return m.T * m.S + m.E + 2; }
 
 // Tensor-core path: tasks hold at most kTcNT tokens (the MMA N), padded to
 // tc_npad rows; a K chunk is 64 packed weight bytes (128 int4 / 256 int2 codes).
-constexpr int kTcNT = 128;
+constexpr int kTcNT = 64;
 __host__ __device__ constexpr int tc_npad(int n) { return n <= 8 ? 8 : (n + 15) & ~15; }
 __host__ __device__ constexpr int tc_kc(int wb) { return 512 / wb; }
 __host__ __device__ constexpr int tc_kpad(int k, int wb) { return (k + tc_kc(wb) - 1) / tc_kc(wb) * tc_kc(wb); }

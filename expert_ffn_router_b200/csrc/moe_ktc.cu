@@ -85,10 +85,20 @@ cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_
     return stage == 0 ? launch_tc_t<2, 0>(p, tm, nt_max, s) : launch_tc_t<2, 1>(p, tm, nt_max, s);
 }
 
+cudaError_t launch_tc_requant(const Params& p, cudaStream_t s) {
+    const int grid = (int)std::min<size_t>((tc_rows_bound(p.m) + kWarps - 1) / kWarps,
+                                           (size_t)persistent_grid((const void*)k_tc_requant<4>, 0));
+    if (p.m.wb == 4) k_tc_requant<4><<<grid, kThreads, 0, s>>>(p);
+    else k_tc_requant<2><<<grid, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tc_gather(const Params& p, const int8_t* src, int ld, int key_div, int K, uint8_t* dst,
                              cudaStream_t s) {
     const int kpad = tc_kpad(K, p.m.wb);
-    const int grid = 2 * persistent_grid((const void*)k_tc_gather<4>, 0);
+    // one warp per padded row; the row count is known on the device only
+    const int grid = (int)std::min<size_t>((tc_rows_bound(p.m) + kWarps - 1) / kWarps,
+                                           (size_t)persistent_grid((const void*)k_tc_gather<4>, 0));
     if (p.m.wb == 4) k_tc_gather<4><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
     else k_tc_gather<2><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
     return cudaGetLastError();

@@ -42,8 +42,10 @@ cudaError_t launch_down(const Params& p, const ExpertTiling& tl, bool dbg, cudaS
 // Tensor-core expert path (moe_ktc.cu).  nt_max: bound on the tokens of one
 // task in this call (<= kTcNT).
 bool tc_shape_ok(const Dims& m);
-// stage 0: gate/up (+ requantisation into the down operand), 1: down.
+// stage 0: gate/up, 1: down.
 cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_t s);
+// h -> the down operand (int8 codes in the MMA layout), scales, code sums.
+cudaError_t launch_tc_requant(const Params& p, cudaStream_t s);
 // Operand B of every task from int8 rows `src` (row = assignment id / key_div).
 cudaError_t launch_tc_gather(const Params& p, const int8_t* src, int ld, int key_div, int K, uint8_t* dst,
                              cudaStream_t s);

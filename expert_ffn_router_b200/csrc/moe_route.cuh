@@ -122,7 +122,8 @@ static __device__ void topk_token(const Params& p, int t, float* s_sm, float* se
 // counts and zero the per-call counters of the expert kernels.  For
 // tensor-core tasks (p.tc) task.w is the task's first row in the padded
 // operand buffers (the sum of tc_npad over the tasks before it).
-// smem: 5 * E ints + kWarps ints.
+// smem: 5 * E + kWarps + kBucketStage ints.
+constexpr int kBucketStage = 1024;  // routing indices staged per pass of the placement
 static __device__ void bucket_cta(const Params& p, int* smem) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = p.m.E, k = p.m.k, T = p.m.T, S = p.m.S, CH = p.CH;
@@ -133,6 +134,7 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     int* off0 = smem + 3 * E;
     int* prow = smem + 4 * E;
     int* red = smem + 5 * E;
+    int* stage = red + kWarps;
     WsHeader* hdr = p.ws.hdr;
     for (int e = tid; e < E; e += kThreads) cnt[e] = 0;
     __syncthreads();
@@ -153,24 +155,33 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     __syncthreads();
     block_exscan(off, E, red);
     const int n_routed_tasks = block_exscan(tb, E, red);
-    if (p.tc) block_exscan(prow, E, red);
+    const int routed_rows = p.tc ? block_exscan(prow, E, red) : 0;
     for (int e = tid; e < E; e += kThreads) off0[e] = off[e];
     __syncthreads();
     const int asg_base = p.m.has_shared ? T : 0;
     const int n_sh_tasks = p.m.has_shared ? (T + CH - 1) / CH : 0;
     const int sh_rows = p.m.has_shared ? (T / CH) * tc_npad(CH) + (T % CH ? tc_npad(T % CH) : 0) : 0;
-    if (warp == 0) {
-        for (int base = 0; base < A; base += 32) {
-            const int a = base + lane;
-            int e = a < A ? __ldcg(p.ws.idx + a) : E;
-            if (e < 0 || e >= E) e = a < A ? 0 : E;
-            const unsigned peers = __match_any_sync(kFull, e);
-            const int rank = __popc(peers & lanemask_lt());
-            if (a < A) p.ws.asg[asg_base + off[e] + rank] = (a / k) * S + (a % k);
-            __syncwarp();
-            if (a < A && rank == 0) off[e] += __popc(peers);
-            __syncwarp();
+    // stable placement by one warp, the indices staged through shared memory
+    for (int base = 0; base < A; base += kBucketStage) {
+        const int nb = min(kBucketStage, A - base);
+        for (int i = tid; i < nb; i += kThreads) {
+            const int e = __ldcg(p.ws.idx + base + i);
+            stage[i] = (e < 0 || e >= E) ? 0 : e;
         }
+        __syncthreads();
+        if (warp == 0) {
+            for (int b = 0; b < nb; b += 32) {
+                const int a = base + b + lane;
+                const int e = b + lane < nb ? stage[b + lane] : E;
+                const unsigned peers = __match_any_sync(kFull, e);
+                const int rank = __popc(peers & lanemask_lt());
+                if (b + lane < nb) p.ws.asg[asg_base + off[e] + rank] = (a / k) * S + (a % k);
+                __syncwarp();
+                if (b + lane < nb && rank == 0) off[e] += __popc(peers);
+                __syncwarp();
+            }
+        }
+        __syncthreads();
     }
     if (p.m.has_shared)
         for (int t = tid; t < T; t += kThreads) p.ws.asg[t] = t * S + k;
@@ -188,6 +199,7 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     for (int i = tid; i < p.nrb4; i += kThreads) p.ws.rb_ctr[i] = 0u;
     if (tid == 0) {
         hdr->n_tasks = n_tasks;
+        hdr->tc_rows = sh_rows + routed_rows;
         hdr->n_asg = T * S;
         hdr->n_items3 = n_tasks * p.nrb3;
         hdr->n_items4 = n_tasks * p.nrb4;
@@ -198,7 +210,7 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
 // 2b+1 for every token (each thread a slice of d, weights streamed once); CTAs
 // b < T also quantise token b.  The last CTA to finish runs the top-k of every
 // token (one warp per token) and, if `bucket`, the bucketing.
-// Dynamic smem: max(2 * kWarps * E floats, 5 * E + kWarps ints).
+// Dynamic smem: max(2 * kWarps * E floats, 5 * E + kWarps + kBucketStage ints).
 template <int TM, int NV, typename XT>
 __global__ void __launch_bounds__(kThreads) k_route_small(const Params p, const XT* __restrict__ x,
                                                           int do_quant, int bucket) {
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(kThreads) k_topk(const Params p) {
     if (t < p.m.T) topk_token(p, t, dsm + warp * 2 * p.m.E, dsm + warp * 2 * p.m.E + p.m.E);
 }
 
-// Bucketing alone (one CTA).  Dynamic smem (5 * E + kWarps) ints.
+// Bucketing alone (one CTA).  Dynamic smem (5 * E + kWarps + kBucketStage) ints.
 __global__ void __launch_bounds__(kThreads) k_bucket(const Params p) {
     extern __shared__ int ism[];
     bucket_cta(p, ism);
@@ -367,6 +379,7 @@ __global__ void __launch_bounds__(kThreads) k_plan_single(const Params p, int bl
     for (int i = threadIdx.x; i < p.nrb4; i += kThreads) p.ws.rb_ctr[i] = 0u;
     if (threadIdx.x == 0) {
         p.ws.hdr->n_tasks = n_tasks;
+        p.ws.hdr->tc_rows = (T / CH) * tc_npad(CH) + (T % CH ? tc_npad(T % CH) : 0);
         p.ws.hdr->n_asg = T;
         p.ws.hdr->n_items3 = n_tasks * p.nrb3;
         p.ws.hdr->n_items4 = n_tasks * p.nrb4;

@@ -15,31 +15,37 @@
 //  B  int8 activations (or requantised h) of the task's tokens, in the
 //     canonical K-major no-swizzle layout of 8-row x 16-byte core matrices,
 //     with each 16-byte K group in the byte order the unpack produces
-//     (permute16).  A gather kernel (x) or the gate/up epilogue (h) writes it
-//     per task and K chunk, so one bulk copy brings a chunk's B into shared
-//     memory.
+//     (permute16).  The gather kernel (x) or the requantisation kernel (h)
+//     writes it per task and K chunk, so one bulk copy brings a chunk's B into
+//     shared memory.
 //
-// Persistent kernel, one CTA per SM, 320 threads:
-//  warp 0    TMA producer: per K chunk two A boxes + the B chunk into a ring
-//            of shared-memory slots (full / empty mbarriers);
-//  warp 1    TMEM allocator and MMA issuer (one thread): per chunk
-//            KC/32 K-steps x 2 tiles, tcgen05.commit releases the slot and the
-//            TMEM A buffer, a final commit per unit hands the accumulators to
-//            the epilogue;
-//  warps 2-9 unpack A into one of two TMEM A buffers, then run the epilogue
-//            (tcgen05.ld of the accumulators).
+// An M = 128, K = 32 MMA costs a fixed ~90 SM cycles for any N <= 128, so one
+// 128-row tile streams at most ~2 packed bytes per cycle per tile; the kernel
+// keeps the MMA pipe issuing back to back.  Persistent, one CTA per SM,
+// 448 threads:
+//  warp 0      TMA producer: per K chunk two A boxes + the B chunk into a
+//              ring of shared-memory slots (full / empty mbarriers);
+//  warp 1      TMEM allocator and MMA issuer (one thread): per chunk
+//              KC/32 K-steps x 2 tiles; tcgen05.commit releases the slot and
+//              the TMEM A buffer, a commit per unit hands an accumulator
+//              buffer to the epilogue;
+//  warps 2-9   unpack A into a ring of TMEM A buffers (two warps per TMEM
+//              lane quarter, each half of a row's chunk);
+//  warps 10-13 epilogue (tcgen05.ld of the accumulators, one warp per lane
+//              quarter), so the MMAs of a unit overlap the previous unit's
+//              epilogue.
 // A unit is (task, row block): two 128-row A tiles sharing one B --
 //  gate/up (EPI 0): gate rows and up rows [128 rb, 128 rb + 128) of f;
-//                   epilogue h = SiLU(g) u, per-token max |h|; the CTA that
-//                   completes a task's last unit requantises the task's h
-//                   into the down operand (hb), its scales and code sums.
+//                   epilogue h = SiLU(g) u and the per-token max |h|
+//                   (requantisation is a separate kernel);
 //  down    (EPI 1): rows [256 rb, 256 rb + 256) of d as two tiles; epilogue
 //                   y = acc (s_row s_h) to the per-assignment buffer (the
 //                   combine is a separate kernel) or straight to the output.
-// TMEM columns: [0, 128) tile-0 accumulators, [128, 256) tile 1, then two A
-// buffers of 2 x KC/4 columns.  Every wait is bounded (kWaitLimitNs); on a
-// timeout the CTA records MOE_ETIMEOUT, lets its copies and MMAs drain and
-// exits.
+// TMEM columns: two accumulator buffers [128 b, 128 b + 128) (tile 0 at
+// +0, tile 1 at +64, N <= 64), then the A buffers from column 256 (2 x KC/4
+// columns each: four for int4, two for int2).  Every wait is bounded
+// (kWaitLimitNs); on a timeout the CTA records MOE_ETIMEOUT, lets its copies
+// and MMAs drain and exits.
 #pragma once
 
 #include <cuda.h>
@@ -48,8 +54,10 @@
 
 namespace moe {
 
-constexpr int kTcThreads = 320;
-constexpr int kTcEpi = 256;                    // unpack / epilogue threads (warps 2-9)
+constexpr int kTcThreads = 448;
+constexpr int kTcUnpack = 256;                 // warps 2-9
+constexpr int kTcEpiWarp0 = 10;                // warps 10-13
+constexpr int kTcEpi = 128;
 constexpr int kTcBox = 128 * 64;               // one A box: 128 rows x 64 packed bytes
 constexpr int kTcSlotA = 2 * kTcBox;           // both tiles of a chunk
 constexpr int kTcMaxSlots = 8;
@@ -57,14 +65,11 @@ constexpr int kTcMaxSlots = 8;
 // Dynamic shared memory: [slots][control block], slots 1024-byte aligned.
 struct TcCtl {
     uint64_t full[kTcMaxSlots], empty[kTcMaxSlots];
-    uint64_t afull[2], afree[2], accfull, accempty, drain;
+    uint64_t afull[4], afree[4], accfull[2], accempty[2], drain;
     uint32_t tmem_base;
-    int last;
-    int asg[2][kTcNT];
-    float sx[2][kTcNT];
-    int cs[2][kTcNT];
-    unsigned amax[kTcNT];
-    int hcs[kTcNT];
+    int asg[kTcNT];
+    float sx[kTcNT];
+    int cs[kTcNT];
 };
 
 __host__ __device__ constexpr int tc_slot_bytes(int nt_max, int wb) {
@@ -137,9 +142,10 @@ __device__ __forceinline__ size_t tc_b_offset(int kg, int j, int npad) {
 template <int WB, int EPI>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_tc(const Params p, const __grid_constant__ CUtensorMap tmA, int ns, int nt_max) {
-    constexpr int KC = tc_kc(WB);         // K columns per chunk
-    constexpr int ACOLS = KC / 4;         // TMEM columns of one tile's A chunk
+    constexpr int KC = tc_kc(WB);           // K columns per chunk
+    constexpr int ACOLS = KC / 4;           // TMEM columns of one tile's A chunk
     constexpr int KSTEPS = KC / 32;
+    constexpr int NAB = 256 / (2 * ACOLS);  // TMEM A buffers
     constexpr int OFF = code_offset<WB>();
     extern __shared__ uint8_t tc_raw[];
     uint8_t* base = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023u)) & 1023u);
@@ -160,18 +166,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&ctl->full[i], 1);
             mbar_init(&ctl->empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->afull[i], kTcEpi);
+        for (int i = 0; i < NAB; ++i) {
+            mbar_init(&ctl->afull[i], kTcUnpack / 32);  // one arrival per unpack warp
             mbar_init(&ctl->afree[i], 1);
         }
-        mbar_init(&ctl->accfull, 1);
-        mbar_init(&ctl->accempty, kTcEpi);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->accfull[i], 1);
+            mbar_init(&ctl->accempty[i], kTcEpi / 32);  // one arrival per epilogue warp
+        }
         mbar_init(&ctl->drain, 1);
         fence_mbar_init();
-    }
-    if (tid >= 64) {
-        ctl->amax[(tid - 64) & (kTcNT - 1)] = 0u;
-        ctl->hcs[(tid - 64) & (kTcNT - 1)] = 0;
     }
     if (warp == 1) tmem_alloc(&ctl->tmem_base, 512);
     tc_fence_before();
@@ -226,20 +230,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int slot = 0;
-            uint32_t ph = 0, g = 0, uidx = 0;
+            int slot = 0, ab = 0;
+            uint32_t ph = 0, abph = 0, uidx = 0;
             bool ok = true, issued = false;
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++uidx) {
                 const int ti = u / nrb;
                 const int npad = tc_npad(p.ws.tasks[ti].z);
                 const uint32_t idesc = tc_idesc_u8s8(npad);
                 const uint32_t lbo = (uint32_t)npad * 16;
-                if (!tc_wait(&ctl->accempty, (uidx & 1u) ^ 1u, hdr, 0x7103)) break;
+                const uint32_t buf = uidx & 1u;
+                const uint32_t dcol = tbase + 128 * buf;
+                if (!tc_wait(&ctl->accempty[buf], ((uidx >> 1) & 1u) ^ 1u, hdr, 0x7103)) break;
                 tc_fence_after();
-                for (int c = 0; c < nch; ++c, ++g) {
-                    const uint32_t ab = g & 1u;
-                    if (!tc_wait(&ctl->full[slot], ph, hdr, 0x7104) ||
-                        !tc_wait(&ctl->afull[ab], (g >> 1) & 1u, hdr, 0x7105)) {
+                for (int c = 0; c < nch; ++c) {
+                    if (!tc_wait(&ctl->full[slot], ph, hdr, 0x7104) || !tc_wait(&ctl->afull[ab], abph, hdr, 0x7105)) {
                         ok = false;
                         break;
                     }
@@ -250,8 +254,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int ks = 0; ks < KSTEPS; ++ks) {
                         const uint64_t bdesc = smem_desc(bsm + ks * 2 * lbo, lbo, 128);
                         const uint32_t acc = (c | ks) != 0;
-                        tc_mma_i8_ts(tbase, acol + ks * 8, bdesc, idesc, acc);
-                        tc_mma_i8_ts(tbase + 128, acol + ACOLS + ks * 8, bdesc, idesc, acc);
+                        tc_mma_i8_ts(dcol, acol + ks * 8, bdesc, idesc, acc);
+                        tc_mma_i8_ts(dcol + 64, acol + ACOLS + ks * 8, bdesc, idesc, acc);
                     }
                     issued = true;
                     tc_commit(&ctl->empty[slot]);
@@ -260,8 +264,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         slot = 0;
                         ph ^= 1u;
                     }
+                    if (++ab == NAB) {
+                        ab = 0;
+                        abph ^= 1u;
+                    }
                 }
-                if (ok) tc_commit(&ctl->accfull);
+                if (ok) tc_commit(&ctl->accfull[buf]);
             }
             // drain: every MMA issued has completed before TMEM is released
             if (issued) {
@@ -269,42 +277,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_wait_bounded(&ctl->drain, 0, hdr, 0x7106);
             }
         }
-    } else {
-        // ------------------------------------------------------------ unpack + epilogue
-        const int etid = tid - 64;
+    } else if (warp < kTcEpiWarp0) {
+        // ------------------------------------------------------------ unpack
+        // A failed wait (timeout, or another wait of the call failed) makes
+        // `ok` false for the whole warp; the warp then skips the tensor-memory
+        // work but still arrives on every mbarrier.
         const int ew = warp - 2;
         const int q = warp & 3;            // TMEM lane quarter this warp may access
-        const int hh = ew >> 2;            // which half of a chunk's units / of the tokens
+        const int hh = ew >> 2;            // which half of a chunk row
         const int row = 32 * q + lane;     // row of the 128-row tiles
         const uint32_t tlane = tbase + ((uint32_t)(32 * q) << 16);
-        // A failed wait (timeout, or another wait of the call failed) makes
-        // `ok` false for the whole warp; the thread then skips the tensor-memory
-        // work but still arrives on every mbarrier and reaches every named
-        // barrier, so no thread of the CTA is left waiting.
-        int slot = 0;
-        uint32_t ph = 0, g = 0, uidx = 0;
+        int slot = 0, ab = 0;
+        uint32_t ph = 0, abph = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++uidx) {
-            const int ti = u / nrb, rb = u - ti * nrb;
-            const int4 task = p.ws.tasks[ti];
-            const int n = task.z, npad = tc_npad(n);
-            const int mb = uidx & 1;
-            if (etid < n) {
-                const int a = p.ws.asg[task.y + etid];
-                ctl->asg[mb][etid] = a;
-                if (EPI == 0) {
-                    const int tok = a / p.m.S;
-                    ctl->sx[mb][etid] = p.ws.sx[tok];
-                    ctl->cs[mb][etid] = p.ws.xcs[tok];
-                } else {
-                    ctl->sx[mb][etid] = p.sh_in ? p.sh_in[a] : __ldcg(p.ws.sh + a);
-                    ctl->cs[mb][etid] = __ldcg(p.ws.hcs + a);
-                }
-            }
-            for (int c = 0; c < nch; ++c, ++g) {
-                const uint32_t ab = g & 1u;
-                if (ok) ok = tc_wait(&ctl->full[slot], ph, hdr, 0x7107) &&
-                             tc_wait(&ctl->afree[ab], ((g >> 1) & 1u) ^ 1u, hdr, 0x7108);
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            for (int c = 0; c < nch; ++c) {
+                if (ok) ok = tc_wait(&ctl->full[slot], ph, hdr, 0x7107) && tc_wait(&ctl->afree[ab], abph ^ 1u, hdr, 0x7108);
                 ok = __all_sync(kFull, ok);
                 if (ok) {
                     tc_fence_after();
@@ -315,34 +303,67 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_st_wait();
                 }
                 tc_fence_before();
-                mbar_arrive(&ctl->afull[ab]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->afull[ab]);
                 if (++slot == ns) {
                     slot = 0;
                     ph ^= 1u;
                 }
+                if (++ab == NAB) {
+                    ab = 0;
+                    abph ^= 1u;
+                }
             }
-            named_sync(1, kTcEpi);  // token metadata of this unit staged
-            if (ok) ok = tc_wait(&ctl->accfull, uidx & 1u, hdr, 0x7109);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int etid = tid - 32 * kTcEpiWarp0;
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        const uint32_t tlane = tbase + ((uint32_t)(32 * q) << 16);
+        uint32_t uidx = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++uidx) {
+            const int ti = u / nrb, rb = u - ti * nrb;
+            const int4 task = p.ws.tasks[ti];
+            const int n = task.z, npad = tc_npad(n);
+            const uint32_t buf = uidx & 1u;
+            named_sync(2, kTcEpi);  // the previous unit's metadata is no longer read
+            if (etid < n) {
+                const int a = p.ws.asg[task.y + etid];
+                ctl->asg[etid] = a;
+                if (EPI == 0) {
+                    const int tok = a / p.m.S;
+                    ctl->sx[etid] = p.ws.sx[tok];
+                    ctl->cs[etid] = p.ws.xcs[tok];
+                } else {
+                    ctl->sx[etid] = p.sh_in ? p.sh_in[a] : __ldcg(p.ws.sh + a);
+                    ctl->cs[etid] = __ldcg(p.ws.hcs + a);
+                }
+            }
+            named_sync(2, kTcEpi);
+            if (ok) ok = tc_wait(&ctl->accfull[buf], (uidx >> 1) & 1u, hdr, 0x7109);
             ok = __all_sync(kFull, ok);
             tc_fence_after();
+            const uint32_t dcol = tlane + 128 * buf;
             if (ok && EPI == 0) {
                 const int r = rb * 128 + row;
                 const bool rv = r < f;
                 const float sg = rv ? __ldg(p.scales + (size_t)task.x * p.scale_rows + r) : 0.0f;
                 const float su = rv ? __ldg(p.scales + (size_t)task.x * p.scale_rows + f + r) : 0.0f;
-                for (int tg = hh; tg * 8 < npad; tg += 2) {
+                for (int tg = 0; tg * 8 < npad; ++tg) {
                     int G[8], U[8];
-                    tmem_ld8(tlane + tg * 8, G);
-                    tmem_ld8(tlane + 128 + tg * 8, U);
+                    tmem_ld8(dcol + tg * 8, G);
+                    tmem_ld8(dcol + 64 + tg * 8, U);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int t = tg * 8 + j;
                         if (t >= n) break;
-                        const int a = ctl->asg[mb][t];
-                        const float sx = ctl->sx[mb][t];
-                        const int gi = G[j] - OFF * ctl->cs[mb][t];
-                        const int ui = U[j] - OFF * ctl->cs[mb][t];
+                        const int a = ctl->asg[t];
+                        const float sx = ctl->sx[t];
+                        const int gi = G[j] - OFF * ctl->cs[t];
+                        const int ui = U[j] - OFF * ctl->cs[t];
                         const float gv = __fmul_rn((float)gi, __fmul_rn(sg, sx));
                         const float uv = __fmul_rn((float)ui, __fmul_rn(su, sx));
                         const float h = __fmul_rn(__fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv))), uv);
@@ -354,7 +375,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             }
                         }
                         const unsigned m = __reduce_max_sync(kFull, rv ? __float_as_uint(fabsf(h)) : 0u);
-                        if (lane == 0) atomicMax(&ctl->amax[t], m);
+                        if (lane == 0 && m != 0u) atomicMax(&p.ws.amax[a], m);
                     }
                 }
             } else if (ok) {
@@ -363,19 +384,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const float s0 = r0 < d ? __ldg(sd + r0) : 0.0f;
                 const float s1 = r0 + 128 < d ? __ldg(sd + r0 + 128) : 0.0f;
                 float* dst = p.direct_out ? p.out : p.ws.ybuf;
-                for (int tg = hh; tg * 8 < npad; tg += 2) {
+                for (int tg = 0; tg * 8 < npad; ++tg) {
                     int D0[8], D1[8];
-                    tmem_ld8(tlane + tg * 8, D0);
-                    tmem_ld8(tlane + 128 + tg * 8, D1);
+                    tmem_ld8(dcol + tg * 8, D0);
+                    tmem_ld8(dcol + 64 + tg * 8, D1);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int t = tg * 8 + j;
                         if (t >= n) break;
-                        const int a = ctl->asg[mb][t];
-                        const float sh = ctl->sx[mb][t];
-                        const int d0 = D0[j] - OFF * ctl->cs[mb][t];
-                        const int d1 = D1[j] - OFF * ctl->cs[mb][t];
+                        const int a = ctl->asg[t];
+                        const float sh = ctl->sx[t];
+                        const int d0 = D0[j] - OFF * ctl->cs[t];
+                        const int d1 = D1[j] - OFF * ctl->cs[t];
                         if (r0 < d) {
                             dst[(size_t)a * d + r0] = __fmul_rn((float)d0, __fmul_rn(s0, sh));
                             if (p.dbg_acc_d) p.dbg_acc_d[(size_t)a * d + r0] = d0;
@@ -388,65 +409,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&ctl->accempty);
-            if (EPI == 0) {
-                named_sync(1, kTcEpi);  // per-token maxima of this CTA complete
-                if (etid < n) {
-                    atomicMax(&p.ws.amax[ctl->asg[mb][etid]], ctl->amax[etid]);
-                    ctl->amax[etid] = 0u;
-                }
-                __threadfence();        // this thread's h stores and maxima before the task count
-                named_sync(1, kTcEpi);
-                if (etid == 0) {
-                    __threadfence();
-                    ctl->last = ok && atomicAdd(&p.ws.task_ctr[ti], 1u) == (unsigned)(nrb - 1);
-                }
-                named_sync(1, kTcEpi);
-                if (ctl->last) {
-                    // every unit of this task is done: requantise its h (a4's
-                    // input rule) into the down operand, in the MMA layout
-                    __threadfence();
-                    if (etid == 0) p.ws.task_ctr[ti] = 0u;
-                    const int npk = tc_kpad(f, WB) / 16;  // 16-column groups per padded row
-                    uint8_t* hb = p.ws.hb + (size_t)task.w * tc_kpad(f, WB);
-                    for (int it = etid; it < npad * npk; it += kTcEpi) {
-                        const int j = it / npk, kg = it - j * npk;
-                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                        if (j < n && kg * 16 < f) {
-                            const int a = ctl->asg[mb][j];
-                            const float m = __uint_as_float(__ldcg(p.ws.amax + a));
-                            if (m != 0.0f) {
-                                const float sh = __fdiv_rn(m, 127.0f);
-                                const float4* hp = reinterpret_cast<const float4*>(p.ws.h + (size_t)a * f + kg * 16);
-                                uint32_t wv[4];
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const float4 hv = __ldcg(hp + i);
-                                    wv[i] = (uint32_t)(quant_code(hv.x, sh) & 0xFF) |
-                                            ((uint32_t)(quant_code(hv.y, sh) & 0xFF) << 8) |
-                                            ((uint32_t)(quant_code(hv.z, sh) & 0xFF) << 16) |
-                                            ((uint32_t)(quant_code(hv.w, sh) & 0xFF) << 24);
-                                }
-                                v = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                            }
-                            atomicAdd(&ctl->hcs[j], sum16(v));
-                            if (p.dbg_hq) *reinterpret_cast<uint4*>(p.dbg_hq + (size_t)a * f + kg * 16) = v;
-                        }
-                        *reinterpret_cast<uint4*>(hb + tc_b_offset(kg, j, npad)) = permute16<WB>(v);
-                    }
-                    named_sync(1, kTcEpi);  // every read of the task's maxima above is done
-                    if (etid < n) {
-                        const int a = ctl->asg[mb][etid];
-                        const float m = __uint_as_float(__ldcg(p.ws.amax + a));
-                        const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-                        p.ws.sh[a] = sh;
-                        p.ws.hcs[a] = ctl->hcs[etid];
-                        if (p.dbg_sh) p.dbg_sh[a] = sh;
-                        ctl->hcs[etid] = 0;
-                        p.ws.amax[a] = 0u;  // leave the workspace's maxima zeroed for the next call
-                    }
-                }
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->accempty[buf]);
         }
     }
     tc_fence_before();
@@ -458,26 +422,88 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
-// Build the gate/up operand B of every task: the int8 rows of the task's
-// tokens (row key = assignment id / key_div of `src`, `ld` bytes apart),
-// K columns [0, K) zero-padded to kpad and rows padded to tc_npad, in the
-// MMA layout with permute16 byte order.
+// a4's input rule on the tensor-core path: requantise each assignment's h
+// (max |h| from the gate/up epilogue) into the down operand B, in the MMA
+// layout, with its scale and code sum; leaves the maxima zeroed.  One warp per
+// padded row of the call, as in the gather.
+template <int WB>
+__global__ void __launch_bounds__(kThreads) k_tc_requant(const Params p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int f = p.m.f;
+    const int n_tasks = p.ws.hdr->n_tasks, rows = p.ws.hdr->tc_rows;
+    const int kpad = tc_kpad(f, WB), npk = kpad / 16;
+    for (int R = blockIdx.x * kWarps + warp; R < rows; R += gridDim.x * kWarps) {
+        int lo = 0, hi = n_tasks - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(&p.ws.tasks[mid].w) <= R) lo = mid;
+            else hi = mid - 1;
+        }
+        const int4 task = __ldg(p.ws.tasks + lo);
+        const int j = R - task.w, npad = tc_npad(task.z);
+        const bool live = j < task.z;
+        const int a = live ? __ldg(p.ws.asg + task.y + j) : 0;
+        const float m = live ? __uint_as_float(__ldcg(p.ws.amax + a)) : 0.0f;
+        const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+        const float* hrow = p.ws.h + (size_t)a * f;
+        uint8_t* out = p.ws.hb + (size_t)task.w * kpad;
+        int cs = 0;
+#pragma unroll 2
+        for (int kg = lane; kg < npk; kg += 32) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (m != 0.0f && kg * 16 < f) {
+                const float4* hp = reinterpret_cast<const float4*>(hrow + kg * 16);
+                uint32_t wv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 hv = __ldcg(hp + i);
+                    wv[i] = (uint32_t)(quant_code(hv.x, sh) & 0xFF) | ((uint32_t)(quant_code(hv.y, sh) & 0xFF) << 8) |
+                            ((uint32_t)(quant_code(hv.z, sh) & 0xFF) << 16) |
+                            ((uint32_t)(quant_code(hv.w, sh) & 0xFF) << 24);
+                }
+                v = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            cs += sum16(v);
+            if (live && p.dbg_hq && kg * 16 < f) *reinterpret_cast<uint4*>(p.dbg_hq + (size_t)a * f + kg * 16) = v;
+            *reinterpret_cast<uint4*>(out + tc_b_offset(kg, j, npad)) = permute16<WB>(v);
+        }
+        cs = __reduce_add_sync(kFull, cs);
+        if (live && lane == 0) {
+            p.ws.sh[a] = sh;
+            p.ws.hcs[a] = cs;
+            if (p.dbg_sh) p.dbg_sh[a] = sh;
+            p.ws.amax[a] = 0u;  // every lane has read it (the reduction above synchronised the warp)
+        }
+    }
+}
+
+// Build the operand B of every task from int8 rows (row key = assignment id /
+// key_div of `src`, `ld` bytes apart): K columns [0, K) zero-padded to kpad,
+// rows padded to tc_npad, in the MMA layout with permute16 byte order.  One
+// warp per padded row of the call (hdr->tc_rows); a row finds its task by
+// binary search over the tasks' first rows (task.w, ascending).
 template <int WB>
 __global__ void __launch_bounds__(kThreads) k_tc_gather(const Params p, const int8_t* __restrict__ src, int ld,
                                                         int key_div, int K, int kpad, uint8_t* __restrict__ dst) {
-    const int n_tasks = p.ws.hdr->n_tasks;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tasks = p.ws.hdr->n_tasks, rows = p.ws.hdr->tc_rows;
     const int npk = kpad / 16;
-    for (int ti = blockIdx.x; ti < n_tasks; ti += gridDim.x) {
-        const int4 task = p.ws.tasks[ti];
-        const int n = task.z, npad = tc_npad(n);
+    for (int R = blockIdx.x * kWarps + warp; R < rows; R += gridDim.x * kWarps) {
+        int lo = 0, hi = n_tasks - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(&p.ws.tasks[mid].w) <= R) lo = mid;
+            else hi = mid - 1;
+        }
+        const int4 task = __ldg(p.ws.tasks + lo);
+        const int j = R - task.w, npad = tc_npad(task.z);
+        const int key = j < task.z ? __ldg(p.ws.asg + task.y + j) / key_div : -1;
+        const int8_t* row = src + (size_t)(key < 0 ? 0 : key) * ld;
         uint8_t* out = dst + (size_t)task.w * kpad;
-        for (int it = threadIdx.x; it < npad * npk; it += kThreads) {
-            const int j = it / npk, kg = it - j * npk;
+#pragma unroll 4
+        for (int kg = lane; kg < npk; kg += 32) {
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (j < n && kg * 16 < K) {
-                const int key = p.ws.asg[task.y + j] / key_div;
-                v = __ldcg(reinterpret_cast<const uint4*>(src + (size_t)key * ld + kg * 16));
-            }
+            if (key >= 0 && kg * 16 < K) v = __ldcg(reinterpret_cast<const uint4*>(row + kg * 16));
             *reinterpret_cast<uint4*>(out + tc_b_offset(kg, j, npad)) = permute16<WB>(v);
         }
     }

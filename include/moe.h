@@ -175,7 +175,7 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *        down kernels on dp4a integer dots), MOE_PATH_DECODE (2: one
  *        persistent kernel for T <= 8; MOE_EINVAL if the shape does not fit
  *        it) or MOE_PATH_TC (3: routing, then gate/up and down as int8
- *        grouped GEMMs on the tensor cores, tasks of up to 128 tokens per
+ *        grouped GEMMs on the tensor cores, tasks of up to 64 tokens per
  *        expert, then the combine).  AUTO takes DECODE where it fits, else TC
  *        when T >= tc_min_tokens, else MULTI.
  *  path_ran: set to the path that ran (MOE_PATH_DECODE, _MULTI or _TC).

@@ -2,7 +2,7 @@
 oracle, through the C ABI.
 
 Forced with moe_config.tc_min_tokens = 1 (or the layer's MOE_PATH_TC).  Cases
-span: padded token counts of 8 and 16 and a multiple of 16, tasks split at 128
+span: padded token counts of 8 and 16 and a multiple of 16, tasks split at 64
 tokens (130, 160, 300 tokens of one expert), ragged K (d = 1056: the last
 128-column chunk is partly outside the row; f = 320 with int2: 256-column
 chunks), ragged rows (f = 352: the last 128-row tile is partly another
@@ -92,7 +92,7 @@ def run_layer_tc(wl, dl, x, accumulate_into=None, ws=None, path=M.MOE_PATH_TC):
     assert_ok(ws)
     if path == M.MOE_PATH_TC:
         assert opts.path_ran == M.MOE_PATH_TC
-        assert opts.n_launches == (1 if T <= 8 else 4) + 4  # router, gather, gate/up, down, combine
+        assert opts.n_launches == (1 if T <= 8 else 4) + 5  # router, gather, gate/up, requant, down, combine
     return out, idx.cpu().numpy(), w.cpu().numpy()
 
 
