@@ -38,12 +38,15 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header must stay 256 bytes");
 
-constexpr int kReadyFlags = 2048;  // per-task ready flags of the decode kernel
+// Decode-kernel control words after the header: [0, 1024) and [1024, 2048)
+// gate/up rows finished per task (the two halves alternate by call parity),
+// [2048, 3072) per-task "requantised h published" flags (epoch valued).
+constexpr int kReadyFlags = 4096;
 constexpr size_t kCtrlBytes = sizeof(WsHeader) + kReadyFlags * 4;  // zeroed by moe_workspace_init
 
 struct Ws {
     WsHeader* hdr;
-    uint32_t* ready;   // [kReadyFlags] epoch at which each task's hq became ready
+    uint32_t* ready;   // [kReadyFlags] decode-kernel per-task counters and flags (see kReadyFlags)
     int8_t* xq;        // [T][d]     quantised activations
     float* sx;         // [T]        activation scales
     int32_t* xcs;      // [T]        sum of each token's codes
@@ -61,6 +64,7 @@ struct Ws {
     float* ybuf;       // [T*S][d]   per-assignment down outputs before the combine
     uint32_t* rb_ctr;  // [ceil(d/rb4)] down item arrivals per row block (self-resetting)
     int32_t* hcs;      // [T*S]      sum of the hq codes of each assignment (tensor-core down)
+    int4* hmeta;       // [T*S]      (scale bits, code sum, -, -) of each assignment's hq (decode down)
     uint8_t* xb;       // tensor-core operand B of gate/up: per task, activation rows in MMA layout
     uint8_t* hb;       // tensor-core operand B of down: per task, hq rows in MMA layout
     size_t bytes;
@@ -124,6 +128,7 @@ inline Ws ws_carve(const Dims& m, void* base) {
     w.ybuf = (float*)take(A * m.d * 4);
     w.rb_ctr = (uint32_t*)take((size_t)((m.d + kMinRowBlock4 - 1) / kMinRowBlock4) * 4);
     w.hcs = (int32_t*)take(A * 4);
+    w.hmeta = (int4*)take(A * 16);
     w.xb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.d, m.wb));
     w.hb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.f, m.wb));
     w.bytes = off;
@@ -263,6 +268,15 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Fire-and-forget add (no value returned to the thread).
+__device__ __forceinline__ void red_add_u32(uint32_t* p, uint32_t v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's earlier global writes before its later ones at GPU scope.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// Orders generic-proxy accesses against async-proxy (bulk copy) accesses of the
+// same memory, e.g. codes stored by one CTA and bulk-copied by another.
+__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 __device__ __forceinline__ int ld_volatile_status(const WsHeader* h) {
     return *reinterpret_cast<const volatile int*>(&h->status);
 }

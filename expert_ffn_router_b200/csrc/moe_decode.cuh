@@ -15,9 +15,16 @@
 //   3. shared-expert gate/up units (need no routing) while the barrier fills;
 //   4. after the barrier every CTA reads all logits and derives the same
 //      top-k routing and the same expert task list (no second barrier);
-//   5. routed gate/up units; the warp that completes a task's last row
-//      requantises its h and publishes the task as ready (release flag);
-//   6. down units (waiting, bounded, for their task's ready flag); at the end
+//   5. routed gate/up units; each warp counts the rows it finished per task
+//      and, once at the end of the phase, publishes the counts (one release
+//      fence, then fire-and-forget adds on per-task counters);
+//   6r. single token: one CTA per task requantises the task's h once (after
+//      the task's counter shows every gate/up row) into int8 codes in the
+//      dot layout and publishes them; every CTA then owns a contiguous range
+//      of output rows, streams those rows of every task's down matrix
+//      together with the task's codes, and combines its rows locally;
+//   6. otherwise: down units (waiting, bounded, until their task's counter
+//      shows every gate/up row) requantise and stage the task's h; at the end
 //      each CTA signs its row blocks off and the CTA bringing a row block's
 //      last task combines it.
 // Each expert selected by several tokens is streamed once: a task is one
@@ -42,6 +49,7 @@ constexpr int kDecMaxK = 32;
 constexpr int kDecMaxTasks = kDecMaxT * kDecMaxK + 1;
 constexpr int kDecBiasCache = 256;  // experts whose bias the kernel keeps in shared memory
 constexpr int kDecBar = 1;  // named barrier of all consumer warps; 2 + g: group g
+constexpr int kDecNQ = 6;   // down rows per warp per unit of the unrolled shapes (rd = 48)
 
 struct DecPlan {
     int slot_bytes, nslot;
@@ -51,7 +59,12 @@ struct DecPlan {
     int nu_gu, nu_dn;  // units per task
     int xs_off, hs_off, ring_off, smem_bytes;
     int hs_grp_bytes;  // h staging bytes of one consumer group (T * f)
+    int rowrange;      // single-token down by output-row ranges (see step 6r)
 };
+// Row-range down unit (single token): [rows x down row][.. hq codes at
+// wbytes - f][row scales at wbytes][(scale, code sum) record at wbytes + 176].
+constexpr int kDecRRMaxRows = 44;
+constexpr int kDecRRMetaOff = 4 * kDecNQ * kDecWarps - 16;
 
 struct DecCtl {
     uint64_t full[kDecMaxSlots];
@@ -296,6 +309,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     // call zeroes the one the next call uses
     uint32_t* amax_cur = (epoch & 1) ? p.ws.amax2 : p.ws.amax;
     uint32_t* amax_nxt = (epoch & 1) ? p.ws.amax : p.ws.amax2;
+    // the same for the per-task counts of finished gate/up rows
+    uint32_t* rows_cur = p.ws.ready + (epoch & 1) * 1024;
+    uint32_t* rows_nxt = p.ws.ready + ((epoch & 1) ^ 1) * 1024;
+    uint32_t* hq_ready = p.ws.ready + 2048;
+    // this CTA's output rows in the row-range down: whole quads of rows, so
+    // the row scales are whole 16-byte bulk copies
+    const int rr_lo = (int)((long long)c * (d / 4) / G) * 4;
+    const int rr_rows = (int)((long long)(c + 1) * (d / 4) / G) * 4 - rr_lo;
+    const bool rowrange = TM == 1 && ND > 0 && pl.rowrange;
     if (tid == 0) DEC_TRACE(0);
     const int n_my_router = c < E ? (E - c + G - 1) / G : 0;  // experts c, c+G, ...
     const int n_router_units = (n_my_router + pl.rr - 1) / pl.rr;
@@ -368,7 +390,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 }
             }
         }
-        {
+        if (rowrange) {
+            // one unit per task: this CTA's rows of the task's down matrix, the
+            // task's published codes and their (scale, code sum) record
+            for (int ti = 0; ti < n_tasks; ++ti) {
+                flag_wait_bounded(hq_ready + ti, epoch + 1, hdr, 130);
+                fence_proxy_async_all();  // the codes were stored by another CTA's threads
+                const int blob = min(max(C.tasks[ti].x, 0), n_blobs - 1);
+                const int a = min(max(C.ttok[ti][0], 0), p.a_cap - 1);
+                uint64_t* bar = &C.full[ps];
+                const uint32_t wb = (uint32_t)rr_rows * rb_dn;
+                uint8_t* dst = take(wb + (uint32_t)f + (uint32_t)rr_rows * 4 + 16);
+                bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)rr_lo * rb_dn, wb,
+                         bar);
+                bulk_g2s(dst + pl.wbytes - f, p.ws.hq + (size_t)a * f, (uint32_t)f, bar);
+                bulk_g2s(dst + pl.wbytes, p.scales + (size_t)blob * p.scale_rows + 2 * f + rr_lo, (uint32_t)rr_rows * 4,
+                         bar);
+                bulk_g2s(dst + pl.wbytes + kDecRRMetaOff, p.ws.hmeta + a, 16, bar);
+                advance();
+            }
+        } else {
             const long long Nd = (long long)n_tasks * pl.nu_dn;
             const long long lo = c * Nd / G, hi = (c + 1) * Nd / G;
             int ti = (int)(lo / pl.nu_dn), j = (int)(lo % pl.nu_dn);
@@ -441,15 +482,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     }
     named_sync(kDecBar, kDecCons);
     if (ctid == 0) DEC_TRACE(1);
-    // single-token decode with the production shape: the lane's activation
-    // chunks stay in registers for every gate/up row
-    uint4 xr[NG > 0 ? NG : 1][NSUB];
-    if (TM == 1 && NG > 0) {
-#pragma unroll
-        for (int i = 0; i < (NG > 0 ? NG : 1); ++i)
-#pragma unroll
-            for (int sb = 0; sb < NSUB; ++sb) xr[i][sb] = xs[sb * nch_gu + lane + 32 * i];
-    }
 
     // unit index (identical sequence to the producer's) and its ring slot and
     // phase, advanced without divisions; unit u belongs to group u & 1
@@ -537,6 +569,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     }
 
     // ---- per-warp gate/up bookkeeping ----
+    // Rows finished per task are counted in registers and published once, at
+    // the end of the gate/up phase: a fence and an atomic with a returned
+    // value per task switch stalled each warp for microseconds while HBM was
+    // saturated.  A warp's units span at most a few tasks; a fifth one
+    // publishes the oldest early.
+    constexpr int kPend = 4;
+    int pend_task[kPend], pend_cnt[kPend], n_pend = 0;
     int cur_task = -1, cur_cnt = 0, cur_n = 0;
     int xoff[TM];    // staged-row offsets (uint4) of the current task's tokens
     int t_asg[TM];   // their assignment ids
@@ -551,21 +590,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         t_cs[i] = 0;
         t_sx[i] = 0.0f;
     }
-    auto flush_gu = [&]() {
+    auto publish = [&](int n_keep) {  // publish all but the newest n_keep pending counts
+        fence_acq_rel_gpu();          // this warp's h stores and maxima before its counts
+        __syncwarp();
+        if (lane == 0)
+            for (int i = 0; i < n_pend - n_keep; ++i) red_add_u32(rows_cur + pend_task[i], (uint32_t)pend_cnt[i]);
+        for (int i = 0; i < n_keep; ++i) {
+            pend_task[i] = pend_task[n_pend - n_keep + i];
+            pend_cnt[i] = pend_cnt[n_pend - n_keep + i];
+        }
+        n_pend = n_keep;
+    };
+    auto flush_gu = [&]() {  // close the current task: maxima now, the row count later
         if (cur_task < 0 || cur_cnt == 0) return;
 #pragma unroll
         for (int i = 0; i < TM; ++i)
             if (i < cur_n && lane == i) atomicMax(amax_cur + t_asg[i], __float_as_uint(amax[i]));
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) {  // the warp bringing the task's last rows publishes it
-            const unsigned t0 = atomicAdd(p.ws.task_ctr + cur_task, (unsigned)cur_cnt);
-            if (t0 + cur_cnt == (unsigned)(pl.nu_gu * kDecWarps)) {
-                p.ws.task_ctr[cur_task] = 0u;
-                __threadfence();
-                st_release_u32(p.ws.ready + cur_task, epoch + 1);
-            }
-        }
+        if (n_pend == kPend) publish(0);
+        pend_task[n_pend] = cur_task;
+        pend_cnt[n_pend] = cur_cnt;
+        ++n_pend;
         cur_cnt = 0;
 #pragma unroll
         for (int i = 0; i < TM; ++i) amax[i] = 0.0f;
@@ -588,9 +632,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         const uint8_t* slot = wait_full();
         const int r = j * kDecWarps + gw;
         const int n = cur_n;
+        bool released = false;
         if (r < f) {
             const uint8_t* grow = slot + (size_t)gw * rb_gu;
             const uint8_t* urow = slot + (size_t)(kDecWarps + gw) * rb_gu;
+            const float* ssc = reinterpret_cast<const float*>(slot + pl.wbytes);
+            float sg, su;
             int ag[TM], au[TM];
 #pragma unroll
             for (int i = 0; i < TM; ++i) ag[i] = au[i] = 0;
@@ -601,12 +648,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     wg[i] = *reinterpret_cast<const uint4*>(grow + (size_t)(lane + 32 * i) * 16);
                     wu[i] = *reinterpret_cast<const uint4*>(urow + (size_t)(lane + 32 * i) * 16);
                 }
+                sg = ssc[gw];
+                su = ssc[kDecWarps + gw];
+                // the warp's rows are in registers: hand the slot back before the dots
+                release();
+                released = true;
                 if constexpr (TM == 1) {
                     int g0 = 0, g1 = 0, u0 = 0, u1 = 0;
 #pragma unroll
                     for (int i = 0; i < NG; ++i) {
-                        dot_chunk_regs<WB>(wg[i], xr[i], g0, g1);
-                        dot_chunk_regs<WB>(wu[i], xr[i], u0, u1);
+                        uint4 xv[NSUB];
+#pragma unroll
+                        for (int sb = 0; sb < NSUB; ++sb) xv[sb] = xs[sb * nch_gu + lane + 32 * i];
+                        dot_chunk_regs<WB>(wg[i], xv, g0, g1);
+                        dot_chunk_regs<WB>(wu[i], xv, u0, u1);
                     }
                     ag[0] = g0 + g1;
                     au[0] = u0 + u1;
@@ -631,9 +686,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                             au[t] = dot_chunk<WB>(wu, xs + xoff[t], nch_gu, cc, au[t]);
                         }
                 }
+                sg = ssc[gw];
+                su = ssc[kDecWarps + gw];
             }
-            const float* ssc = reinterpret_cast<const float*>(slot + pl.wbytes);
-            const float sg = ssc[gw], su = ssc[kDecWarps + gw];
 #pragma unroll
             for (int i = 0; i < TM; ++i)
                 if (i < n) {
@@ -648,7 +703,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     }
                 }
         }
-        release();
+        if (!released) release();
         ++cur_cnt;
     };
 
@@ -668,6 +723,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     if (ctid == 0) DEC_TRACE(4);
     if (c == 0 && ctid == 0) hdr->epoch = epoch + 1;
     for (int i = c * kDecCons + ctid; i < p.a_cap; i += G * kDecCons) amax_nxt[i] = 0u;
+    for (int i = c * kDecCons + ctid; i < kDecMaxTasks; i += G * kDecCons) rows_nxt[i] = 0u;
     if (warp < T) {
         int my_e;
         float my_w;
@@ -754,8 +810,106 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             }
         }
         flush_gu();
+        publish(0);
     }
     if (ctid == 0) DEC_TRACE(6);
+
+    // ---- 6r. single token: row-range down with a local combine ----
+    if constexpr (TM == 1 && ND > 0) {
+        if (rowrange) {
+            // requantise the tasks this CTA is designated for (task ti -> CTA ti % G)
+            for (int ti = c; ti < n_tasks; ti += G) {
+                if (ctid == 0) flag_wait_bounded(rows_cur + ti, (uint32_t)(pl.nu_gu * kDecWarps), hdr, 410);
+                named_sync(kDecBar, kDecCons);
+                __threadfence();  // the other CTAs' h rows and maxima
+                const int a = min(max(C.ttok[ti][0], 0), p.a_cap - 1);
+                const float m = __uint_as_float(__ldcg(amax_cur + a));
+                const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+                int cs = 0;
+                if (ctid < f / 16) {
+                    const int pc = ctid;
+                    const float* hrow = p.ws.h + (size_t)a * f;
+                    unsigned wds[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 hv = __ldcg(reinterpret_cast<const float4*>(hrow + pc * 16 + 4 * q4));
+                        const float hs4[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int code = m == 0.0f ? 0 : quant_code(hs4[q], sh);
+                            cs += code;
+                            wds[q4] |= ((unsigned)code & 0xFFu) << (8 * q);
+                        }
+                    }
+                    reinterpret_cast<uint4*>(p.ws.hq + (size_t)a * f)[(pc % NSUB) * nch_dn + pc / NSUB] =
+                        permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
+                    __threadfence();           // the codes before the publication below
+                    fence_proxy_async_all();   // ... and visible to bulk copies
+                }
+                cs = cons_sum_int(cs, C.redi);
+                if (ctid == 0) {
+                    p.ws.hmeta[a] = make_int4(__float_as_int(sh), cs, 0, 0);
+                    __threadfence();
+                    fence_proxy_async_all();  // the codes are read by bulk copies
+                    st_release_u32(hq_ready + ti, epoch + 1);
+                }
+            }
+            if (ctid == 0) DEC_TRACE(7);
+            // down units: one per task, this CTA's rows; y of (assignment, row)
+            // kept in shared memory for the combine
+            float* ys = reinterpret_cast<float*>(hsb);  // [S][kDecNQ * kDecWarps]
+            constexpr int RRW = kDecNQ * kDecWarps;
+            for (int ti = 0; ti < n_tasks; ++ti, next_unit()) {
+                if (!mine()) continue;
+                const uint8_t* slot = wait_full();
+                uint4 hrr[ND][NSUB];
+                const uint4* hq4 = reinterpret_cast<const uint4*>(slot + pl.wbytes - f);
+#pragma unroll
+                for (int i = 0; i < ND; ++i)
+#pragma unroll
+                    for (int sb = 0; sb < NSUB; ++sb) hrr[i][sb] = hq4[sb * nch_dn + lane + 32 * i];
+                const int4 meta = *reinterpret_cast<const int4*>(slot + pl.wbytes + kDecRRMetaOff);
+                const float* sd = reinterpret_cast<const float*>(slot + pl.wbytes);
+                uint4 wv[kDecNQ][ND];
+                float sdr[kDecNQ];
+#pragma unroll
+                for (int q = 0; q < kDecNQ; ++q) {
+                    const int rl = q * kDecWarps + gw;
+                    const bool ok = rl < rr_rows;
+#pragma unroll
+                    for (int i = 0; i < ND; ++i)
+                        wv[q][i] = ok ? *reinterpret_cast<const uint4*>(slot + (size_t)rl * rb_dn + (size_t)(lane + 32 * i) * 16)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+                    sdr[q] = ok ? sd[rl] : 0.0f;
+                }
+                release();
+                const float shv = __int_as_float(meta.x);
+                const int a = min(max(C.ttok[ti][0], 0), S - 1);
+#pragma unroll
+                for (int q = 0; q < kDecNQ; ++q) {
+                    int a0 = 0, a1 = 0;
+#pragma unroll
+                    for (int i = 0; i < ND; ++i) dot_chunk_regs<WB>(wv[q][i], hrr[i], a0, a1);
+                    const int D = __reduce_add_sync(kFull, a0 + a1) - code_offset<WB>() * meta.y;
+                    const int rl = q * kDecWarps + gw;
+                    if (lane == 0 && rl < rr_rows) ys[a * RRW + rl] = __fmul_rn((float)D, __fmul_rn(sdr[q], shv));
+                }
+            }
+            named_sync(kDecBar, kDecCons);  // every y of this CTA's rows is in shared memory
+            for (int rl = ctid; rl < rr_rows; rl += kDecCons) {
+                float o = 0.0f;
+                for (int jj = 0; jj < k; ++jj) o = fmaf(C.w[0][jj], ys[jj * RRW + rl], o);
+                if (HS) o += ys[k * RRW + rl];
+                float* dst = p.out + rr_lo + rl;
+                *dst = p.accumulate ? *dst + o : o;
+            }
+            if (ctid == 0) {
+                DEC_TRACE(8);
+                if (trace) trace[9] = t_full;
+            }
+            return;
+        }
+    }
 
     // ---- 6. down units ----
     uint8_t* hsg = hsb + (size_t)grp * hs_grp;  // this group's staged h codes
@@ -773,7 +927,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         const int n = C.tasks[ti].y;
         if (ti != C.hq_task[grp]) {  // requantise and stage this task's h (the whole group agrees on ti)
             named_sync(2 + grp, kDecGrp);
-            if (gtid == 0) flag_wait_bounded(p.ws.ready + ti, epoch + 1, hdr, 400);
+            if (gtid == 0) flag_wait_bounded(rows_cur + ti, (uint32_t)(pl.nu_gu * kDecWarps), hdr, 400);
             named_sync(2 + grp, kDecGrp);
             for (int i = 0; i < n; ++i) {
                 const int a = C.ttok[ti][i];
@@ -818,6 +972,39 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         const uint8_t* slot = wait_full();
         const float* sd = reinterpret_cast<const float*>(slot + pl.wbytes);  // this unit's row scales
         const int nq = pl.rd / kDecWarps;
+        if constexpr (TM == 1 && ND > 0) {
+            // single token: the warp's kDecNQ rows into registers, the slot back
+            // to the producer, then independent dot chains per row
+            uint4 wv[kDecNQ][ND];
+            float sdr[kDecNQ];
+#pragma unroll
+            for (int q = 0; q < kDecNQ; ++q) {
+                const int rl = q * kDecWarps + gw;
+                const bool ok = j * pl.rd + rl < d;
+#pragma unroll
+                for (int i = 0; i < ND; ++i)
+                    wv[q][i] = ok ? *reinterpret_cast<const uint4*>(slot + (size_t)rl * rb_dn + (size_t)(lane + 32 * i) * 16)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+                sdr[q] = ok ? sd[rl] : 0.0f;
+            }
+            release();
+            int dv[kDecNQ];
+#pragma unroll
+            for (int q = 0; q < kDecNQ; ++q) {
+                int a0 = 0, a1 = 0;
+#pragma unroll
+                for (int i = 0; i < ND; ++i) dot_chunk_regs<WB>(wv[q][i], hr[i], a0, a1);
+                dv[q] = a0 + a1;
+            }
+            const int a = C.ttok[ti][0];
+#pragma unroll
+            for (int q = 0; q < kDecNQ; ++q) {
+                const int D = __reduce_add_sync(kFull, dv[q]) - code_offset<WB>() * C.hcs[grp][0];
+                const int r = j * pl.rd + q * kDecWarps + gw;
+                if (lane == q && r < d) p.ws.ybuf[(size_t)a * d + r] = __fmul_rn((float)D, __fmul_rn(sdr[q], C.hsh[grp][0]));
+            }
+            continue;
+        }
         for (int q = 0; q < nq; ++q) {
             const int rl = q * kDecWarps + gw, r = j * pl.rd + rl;
             if (r >= d) break;

@@ -38,6 +38,14 @@ bool decode_plan(const Dims& m, DecPlan* pl) {
     // ahead, where a parity wait cannot tell the phases apart)
     q.nslot = std::min(kDecMaxSlots, room / slot) / 2 * 2;
     if (q.nslot < 2) return false;
+    // single-token down by output-row ranges: every CTA's rows (whole quads)
+    // of one task fit a unit next to the task's codes, and the per-row outputs
+    // of all assignments fit the h staging area
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int rr_rows_max = sms > 0 ? (m.d / 4 + sms - 1) / sms * 4 : 1 << 30;
+    q.rowrange = m.T == 1 && m.d % 4 == 0 && q.rd == kDecNQ * kDecWarps && rr_rows_max <= kDecRRMaxRows &&
+                 rr_rows_max * rb_dn <= wbytes - m.f && (size_t)m.S * kDecNQ * kDecWarps * 4 <= (size_t)hs;
     q.xs_off = ctl;
     q.hs_off = ctl + xs;
     q.ring_off = ctl + xs + hs;
@@ -78,7 +86,7 @@ template <int WB, typename XT>
 static cudaError_t by_shape(const Params& p, const DecPlan& pl, const void* x, cudaStream_t s) {
     const int nch_gu = p.m.d * WB / 8 / 16, nch_dn = p.m.f * WB / 8 / 16;
     constexpr int NG = WB == 4 ? 6 : 3, ND = WB == 4 ? 2 : 1;
-    if (nch_gu == 32 * NG && nch_dn == 32 * ND) return by_t<WB, NG, ND, XT>(p, pl, x, s);
+    if (nch_gu == 32 * NG && nch_dn == 32 * ND && pl.rd == kDecNQ * kDecWarps) return by_t<WB, NG, ND, XT>(p, pl, x, s);
     return by_t<WB, 0, 0, XT>(p, pl, x, s);
 }
 
