@@ -40,22 +40,29 @@ static unsigned long long cache_key(int dev, const void* func, size_t smem) {
            (unsigned long long)dev;
 }
 
-int persistent_grid(const void* func, size_t smem) {
+// Resident CTAs per SM of a kernel for a block size and dynamic shared memory
+// (cached: the occupancy query costs microseconds of host time).
+int blocks_per_sm(const void* func, size_t smem, int threads) {
     int dev = 0;
     cudaGetDevice(&dev);
-    const unsigned long long key = cache_key(dev, func, smem);
+    const unsigned long long key = cache_key(dev, func, smem) ^ ((unsigned long long)threads << 48);
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_grid.find(key);
         if (it != g_grid.end()) return it->second;
     }
-    int sms = 0, per_sm = 0;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, kThreads, smem);
-    const int grid = std::max(1, sms * std::max(1, per_sm));
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, threads, smem) != cudaSuccess) per_sm = 0;
     std::lock_guard<std::mutex> lk(g_mu);
-    g_grid[key] = grid;
-    return grid;
+    g_grid[key] = per_sm;
+    return per_sm;
+}
+
+int persistent_grid(const void* func, size_t smem, int threads) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return std::max(1, sms * std::max(1, blocks_per_sm(func, smem, threads)));
 }
 
 cudaError_t allow_smem(const void* func, size_t smem) {

@@ -9,21 +9,23 @@
 // on an mbarrier per slot).  The consumers work through the same unit
 // sequence, the two consumer groups taking alternate units (4 warps per
 // scheduler to hide the dot products' latencies):
-//   1. quantise the T tokens (every CTA, into its own shared memory);
-//   2. router units: logits of this CTA's experts -> workspace; arrive at the
-//      one grid barrier;
-//   3. shared-expert gate/up units (need no routing) while the barrier fills;
-//   4. after the barrier every CTA reads all logits and derives the same
+//   1. router units: logits of this CTA's experts (from x as given), turned
+//      at once into (selection value, score) pairs -> workspace; arrive at
+//      the one grid barrier;
+//   2. quantise the T tokens (every CTA, into its own shared memory) and run
+//      the shared expert's gate/up units (need no routing) while the
+//      barrier fills;
+//   3. after the barrier every CTA reads all pairs and derives the same
 //      top-k routing and the same expert task list (no second barrier);
-//   5. routed gate/up units; each warp counts the rows it finished per task
+//   4. routed gate/up units; each warp counts the rows it finished per task
 //      and, once at the end of the phase, publishes the counts (one release
 //      fence, then fire-and-forget adds on per-task counters);
-//   6r. single token: one CTA per task requantises the task's h once (after
+//   5r. single token: one CTA per task requantises the task's h once (after
 //      the task's counter shows every gate/up row) into int8 codes in the
 //      dot layout and publishes them; every CTA then owns a contiguous range
 //      of output rows, streams those rows of every task's down matrix
 //      together with the task's codes, and combines its rows locally;
-//   6. otherwise: down units (waiting, bounded, until their task's counter
+//   5. otherwise: down units (waiting, bounded, until their task's counter
 //      shows every gate/up row) requantise and stage the task's h; at the end
 //      each CTA signs its row blocks off and the CTA bringing a row block's
 //      last task combines it.
@@ -50,6 +52,7 @@ constexpr int kDecMaxTasks = kDecMaxT * kDecMaxK + 1;
 constexpr int kDecBiasCache = 256;  // experts whose bias the kernel keeps in shared memory
 constexpr int kDecBar = 1;  // named barrier of all consumer warps; 2 + g: group g
 constexpr int kDecNQ = 6;   // down rows per warp per unit of the unrolled shapes (rd = 48)
+constexpr int kDecXr = 8;   // router float4 inputs per thread for one token (d <= 8 * 4 * 256)
 
 struct DecPlan {
     int slot_bytes, nslot;
@@ -66,9 +69,12 @@ struct DecPlan {
 constexpr int kDecRRMaxRows = 44;
 constexpr int kDecRRMetaOff = 4 * kDecNQ * kDecWarps - 16;
 
+constexpr int kDecRRMaxTasks = kDecMaxK + 1;  // tasks of a single token (row-range down)
+
 struct DecCtl {
     uint64_t full[kDecMaxSlots];
     uint64_t empty[kDecMaxSlots];
+    uint64_t codes[kDecRRMaxTasks];  // row-range down: task ti's codes landed in its unit's slot
     uint64_t route_ready;
     uint32_t epoch;
     int n_tasks;
@@ -165,16 +171,24 @@ __device__ __forceinline__ void load16(const XT* x, size_t i, float v[16]) {
     }
 }
 
-// Top-k of one token by one warp from a logits row in global memory; lane j
-// (< k) returns slot j's expert and weight.  Same rule as topk_token.
-__device__ __forceinline__ void topk_warp(const float* lrow, const float* bias, int E, int k, float scale,
-                                          float* s_sm, float* sel_sm, int& my_e, float& my_w) {
+// Router output of one (token, expert) as the decode kernel keeps it: the
+// selection value sigmoid(logit) + bias and the score sigmoid(logit), fp32
+// bits, computed by the CTA that owns the expert's router row.
+__device__ __forceinline__ uint2 route_pair(float logit, float bias) {
+    const float s = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-logit)));
+    return make_uint2(__float_as_uint(__fadd_rn(s, bias)), __float_as_uint(s));
+}
+
+// Top-k of one token by one warp from its row of (selection, score) pairs in
+// global memory; lane j (< k) returns slot j's expert and weight.  Same rule
+// as topk_token.
+__device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float scale, float* s_sm, float* sel_sm,
+                                          int& my_e, float& my_w) {
     const int lane = threadIdx.x & 31;
     for (int e = lane; e < E; e += 32) {
-        const float lg = __ldcg(lrow + e);
-        const float s = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-lg)));
-        s_sm[e] = s;
-        sel_sm[e] = __fadd_rn(s, __ldg(bias + e));
+        const uint2 pr = __ldcg(prow + e);
+        s_sm[e] = __uint_as_float(pr.y);
+        sel_sm[e] = __uint_as_float(pr.x);
     }
     __syncwarp();
     float ssum = 0.0f, my_s = 0.0f;
@@ -223,21 +237,18 @@ __device__ __forceinline__ unsigned float_key(float v) {
 // Top-k of one token by one warp for E <= 256: lane l holds experts l + 32 i
 // in registers; each round takes the largest selection score (lowest index on
 // ties) with two warp reductions.  Same rule and arithmetic as topk_warp.
-__device__ __forceinline__ void topk_warp_small(const float* lrow, const float* bias_s, int E, int k, float scale,
-                                                int& my_e, float& my_w) {
+__device__ __forceinline__ void topk_warp_small(const uint2* prow, int E, int k, float scale, int& my_e,
+                                                float& my_w) {
     const int lane = threadIdx.x & 31;
     float sv[8];
     unsigned key[8];
+    uint2 pr[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pr[i] = lane + 32 * i < E ? __ldcg(prow + lane + 32 * i) : make_uint2(0u, 0u);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        sv[i] = 0.0f;
-        key[i] = 0u;  // below every real key
-        if (e < E) {
-            const float lg = __ldcg(lrow + e);
-            sv[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-lg)));
-            key[i] = float_key(__fadd_rn(sv[i], bias_s[e]));
-        }
+        sv[i] = __uint_as_float(pr[i].y);
+        key[i] = lane + 32 * i < E ? float_key(__uint_as_float(pr[i].x)) : 0u;  // 0: below every real key
     }
     float ssum = 0.0f, my_s = 0.0f;
     my_e = 0;
@@ -299,6 +310,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             mbar_init(&C.empty[i], kDecWarps);
         }
         mbar_init(&C.route_ready, 1);
+        for (int i = 0; i < kDecRRMaxTasks; ++i) mbar_init(&C.codes[i], 1);
         fence_mbar_init();
         C.epoch = __ldcg(&hdr->epoch);
         for (int g = 0; g < kDecGroups; ++g) C.hq_task[g] = -1;
@@ -391,24 +403,61 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             }
         }
         if (rowrange) {
-            // one unit per task: this CTA's rows of the task's down matrix, the
-            // task's published codes and their (scale, code sum) record
-            for (int ti = 0; ti < n_tasks; ++ti) {
-                flag_wait_bounded(hq_ready + ti, epoch + 1, hdr, 130);
-                fence_proxy_async_all();  // the codes were stored by another CTA's threads
+            // one unit per task: this CTA's rows of the task's down matrix and
+            // their scales at once; the task's published codes and (scale,
+            // code sum) record follow into the same slot, counted on
+            // C.codes[ti], as soon as the task's flag is seen -- serviced
+            // while waiting for slots, so the weights never wait for the codes
+            uint8_t* dsts[kDecRRMaxTasks];
+            int next_code = 0;
+            auto issue_codes = [&](int n_units) {  // the codes of every published task in order
+                while (next_code < n_units && ld_acquire_u32(hq_ready + next_code) == epoch + 1) {
+                    fence_proxy_async_all();  // the codes were stored by another CTA's threads
+                    const int a = min(max(C.ttok[next_code][0], 0), p.a_cap - 1);
+                    mbar_arrive_expect_tx(&C.codes[next_code], (uint32_t)f + 16);
+                    bulk_g2s(dsts[next_code] + pl.wbytes - f, p.ws.hq + (size_t)a * f, (uint32_t)f, &C.codes[next_code]);
+                    bulk_g2s(dsts[next_code] + pl.wbytes + kDecRRMetaOff, p.ws.hmeta + a, 16, &C.codes[next_code]);
+                    ++next_code;
+                }
+            };
+            const int n_rr = min(n_tasks, kDecRRMaxTasks);
+            for (int ti = 0; ti < n_rr; ++ti) {
+                if (pr > 0) {  // wait for the slot, servicing published codes meanwhile
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(&C.empty[ps], (pr - 1) & 1)) {
+                        issue_codes(ti);
+                        if (global_timer_ns() - t0 > kWaitLimitNs) {
+                            set_status(hdr, MOE_ETIMEOUT, 131);
+                            break;
+                        }
+                    }
+                }
                 const int blob = min(max(C.tasks[ti].x, 0), n_blobs - 1);
-                const int a = min(max(C.ttok[ti][0], 0), p.a_cap - 1);
                 uint64_t* bar = &C.full[ps];
                 const uint32_t wb = (uint32_t)rr_rows * rb_dn;
-                uint8_t* dst = take(wb + (uint32_t)f + (uint32_t)rr_rows * 4 + 16);
+                mbar_arrive_expect_tx(bar, wb + (uint32_t)rr_rows * 4);
+                uint8_t* dst = ring + (size_t)ps * slot_bytes;
+                dsts[ti] = dst;
                 bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)rr_lo * rb_dn, wb,
                          bar);
-                bulk_g2s(dst + pl.wbytes - f, p.ws.hq + (size_t)a * f, (uint32_t)f, bar);
                 bulk_g2s(dst + pl.wbytes, p.scales + (size_t)blob * p.scale_rows + 2 * f + rr_lo, (uint32_t)rr_rows * 4,
                          bar);
-                bulk_g2s(dst + pl.wbytes + kDecRRMetaOff, p.ws.hmeta + a, 16, bar);
                 advance();
+                issue_codes(ti + 1);
             }
+            {  // the codes still unpublished: wait for them in order (bounded)
+                const uint64_t t0 = global_timer_ns();
+                while (next_code < n_rr) {
+                    issue_codes(n_rr);
+                    if (next_code < n_rr && ld_volatile_status(hdr) != 0) break;
+                    if (global_timer_ns() - t0 > kWaitLimitNs) {
+                        set_status(hdr, MOE_ETIMEOUT, 132);
+                        break;
+                    }
+                }
+            }
+            // every code copy issued has landed before the CTA can retire
+            for (int ti = 0; ti < next_code; ++ti) mbar_wait_bounded(&C.codes[ti], 0, hdr, 133);
         } else {
             const long long Nd = (long long)n_tasks * pl.nu_dn;
             const long long lo = c * Nd / G, hi = (c + 1) * Nd / G;
@@ -447,41 +496,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     const int grp = warp / kDecWarps, gw = warp % kDecWarps, gtid = ctid % kDecGrp;
     const int hs_grp = pl.hs_grp_bytes;  // staging bytes of one group
 
-    // ---- 1. quantise the T tokens into the permuted staging layout ----
-    if (E <= kDecBiasCache)
-        for (int e = ctid; e < E; e += kDecCons) C.bias_s[e] = __ldg(p.bias + e);
-    for (int t = 0; t < T; ++t) {
-        const XT* xt = x + (size_t)t * d;
-        float v[16];
-        float m = 0.0f;
-        const int pc = ctid;  // d / 16 <= kDecCons pieces of 16 values
-        if (pc < d / 16) {
-            load16(xt, (size_t)pc * 16, v);
+    // single token: this thread's router inputs x[4v .. 4v + 3], v = gtid + i * kDecGrp
+    float4 xrr[TM == 1 ? kDecXr : 1];
+    if constexpr (TM == 1) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) m = fmaxf(m, fabsf(v[q]));
-        }
-        m = cons_max(m, C.redf);
-        const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-        int cs = 0;
-        if (pc < d / 16) {
-            unsigned wds[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int code = m == 0.0f ? 0 : quant_code(v[q], s);
-                cs += code;
-                wds[q >> 2] |= ((unsigned)code & 0xFFu) << (8 * (q & 3));
-            }
-            xs[(size_t)t * NSUB * nch_gu + (pc % NSUB) * nch_gu + pc / NSUB] =
-                permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
-        }
-        cs = cons_sum_int(cs, C.redi);
-        if (ctid == 0) {
-            C.sx[t] = s;
-            C.xcs[t] = cs;
+        for (int i = 0; i < kDecXr; ++i) {
+            const int v = (ctid % kDecGrp) + i * kDecGrp;
+            xrr[i] = v < d / 4 ? load_x4(x, (size_t)4 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
-    named_sync(kDecBar, kDecCons);
-    if (ctid == 0) DEC_TRACE(1);
+    // ---- 1. the router bias into shared memory (the router reads x as given) ----
+    if (E <= kDecBiasCache)
+        for (int e = ctid; e < E; e += kDecCons) C.bias_s[e] = __ldg(p.bias + e);
+    named_sync(kDecBar, kDecCons);  // the bias cache is filled
 
     // unit index (identical sequence to the producer's) and its ring slot and
     // phase, advanced without divisions; unit u belongs to group u & 1
@@ -519,6 +546,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         for (int i = 0; i < 2; ++i)
 #pragma unroll
             for (int t = 0; t < TM; ++t) acc[i][t] = 0.0f;
+        if constexpr (TM == 1) {  // the token's values were loaded into registers at the start
+#pragma unroll
+            for (int i = 0; i < kDecXr; ++i) {
+                const int v = gtid + i * kDecGrp;
+                if (v < d / 4) {
+                    const float4 w0 = reinterpret_cast<const float4*>(wrow)[v];
+                    const float4 w1 = rows > 1 ? reinterpret_cast<const float4*>(wrow + d)[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    acc[0][0] = fmaf(w0.x, xrr[i].x, acc[0][0]);
+                    acc[0][0] = fmaf(w0.y, xrr[i].y, acc[0][0]);
+                    acc[0][0] = fmaf(w0.z, xrr[i].z, acc[0][0]);
+                    acc[0][0] = fmaf(w0.w, xrr[i].w, acc[0][0]);
+                    acc[1][0] = fmaf(w1.x, xrr[i].x, acc[1][0]);
+                    acc[1][0] = fmaf(w1.y, xrr[i].y, acc[1][0]);
+                    acc[1][0] = fmaf(w1.z, xrr[i].z, acc[1][0]);
+                    acc[1][0] = fmaf(w1.w, xrr[i].w, acc[1][0]);
+                }
+            }
+        } else
         for (int v = gtid; v < d / 4; v += kDecGrp) {
             float4 wv[2];
             wv[0] = reinterpret_cast<const float4*>(wrow)[v];
@@ -551,7 +596,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
 #pragma unroll
             for (int w = 0; w < kDecWarps; ++w) v += C.part[grp][w][i * TM + t];
             const int e = c + (ru * pl.rr + i) * G;
-            p.ws.logits[(size_t)t * E + e] = v;
+            reinterpret_cast<uint2*>(p.ws.logits)[(size_t)t * E + e] =
+                route_pair(v, E <= kDecBiasCache ? C.bias_s[e] : __ldg(p.bias + e));
         }
         named_sync(2 + grp, kDecGrp);
     }
@@ -567,6 +613,41 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             st_release_u32(&hdr->b1_gen, epoch + 1);
         }
     }
+
+    // ---- 2b. quantise the T tokens into the permuted staging layout (while the
+    //          grid barrier fills) ----
+    for (int t = 0; t < T; ++t) {
+        const XT* xt = x + (size_t)t * d;
+        float v[16];
+        float m = 0.0f;
+        const int pc = ctid;  // d / 16 <= kDecCons pieces of 16 values
+        if (pc < d / 16) {
+            load16(xt, (size_t)pc * 16, v);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) m = fmaxf(m, fabsf(v[q]));
+        }
+        m = cons_max(m, C.redf);
+        const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+        int cs = 0;
+        if (pc < d / 16) {
+            unsigned wds[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int code = m == 0.0f ? 0 : quant_code(v[q], s);
+                cs += code;
+                wds[q >> 2] |= ((unsigned)code & 0xFFu) << (8 * (q & 3));
+            }
+            xs[(size_t)t * NSUB * nch_gu + (pc % NSUB) * nch_gu + pc / NSUB] =
+                permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
+        }
+        cs = cons_sum_int(cs, C.redi);
+        if (ctid == 0) {
+            C.sx[t] = s;
+            C.xcs[t] = cs;
+        }
+    }
+    named_sync(kDecBar, kDecCons);
+    if (ctid == 0) DEC_TRACE(1);
 
     // ---- per-warp gate/up bookkeeping ----
     // Rows finished per task are counted in registers and published once, at
@@ -728,10 +809,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         int my_e;
         float my_w;
         if (E <= kDecBiasCache) {
-            topk_warp_small(p.ws.logits + (size_t)warp * E, C.bias_s, E, k, p.routed_scale, my_e, my_w);
+            topk_warp_small(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale,
+                            my_e, my_w);
         } else {
             float* scr = reinterpret_cast<float*>(hsb) + (size_t)warp * 2 * E;
-            topk_warp(p.ws.logits + (size_t)warp * E, p.bias, E, k, p.routed_scale, scr, scr + E, my_e, my_w);
+            topk_warp(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale, scr,
+                      scr + E, my_e, my_w);
         }
         if (lane < k) {
             C.idx[warp][lane] = my_e;
@@ -843,15 +926,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     }
                     reinterpret_cast<uint4*>(p.ws.hq + (size_t)a * f)[(pc % NSUB) * nch_dn + pc / NSUB] =
                         permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
-                    __threadfence();           // the codes before the publication below
-                    fence_proxy_async_all();   // ... and visible to bulk copies
                 }
-                cs = cons_sum_int(cs, C.redi);
+                cs = cons_sum_int(cs, C.redi);  // its barrier orders every thread's codes before thread 0's fence
                 if (ctid == 0) {
                     p.ws.hmeta[a] = make_int4(__float_as_int(sh), cs, 0, 0);
                     __threadfence();
-                    fence_proxy_async_all();  // the codes are read by bulk copies
-                    st_release_u32(hq_ready + ti, epoch + 1);
+                    st_release_u32(hq_ready + ti, epoch + 1);  // readers fence the async proxy before copying
                 }
             }
             if (ctid == 0) DEC_TRACE(7);
@@ -859,9 +939,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             // kept in shared memory for the combine
             float* ys = reinterpret_cast<float*>(hsb);  // [S][kDecNQ * kDecWarps]
             constexpr int RRW = kDecNQ * kDecWarps;
-            for (int ti = 0; ti < n_tasks; ++ti, next_unit()) {
+            for (int ti = 0; ti < min(n_tasks, kDecRRMaxTasks); ++ti, next_unit()) {
                 if (!mine()) continue;
                 const uint8_t* slot = wait_full();
+                mbar_wait_bounded(&C.codes[ti], 0, hdr, 420);
                 uint4 hrr[ND][NSUB];
                 const uint4* hq4 = reinterpret_cast<const uint4*>(slot + pl.wbytes - f);
 #pragma unroll

@@ -1,17 +1,40 @@
 // Instantiations, shared-memory plan and cooperative launch of the persistent
 // decode kernel.
 #include <algorithm>
+#include <mutex>
 
 #include "moe_decode.cuh"
 #include "moe_launch.h"
 
 namespace moe {
 
+// Per-device facts the plan and the launch need, queried once per device.
+struct DevFacts {
+    int optin = 0, sms = 0;
+};
+static std::mutex g_dev_mu;
+static DevFacts g_dev[64];
+static bool dev_facts(DevFacts* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevFacts& f = g_dev[dev];
+    if (f.sms == 0) {
+        if (cudaDeviceGetAttribute(&f.optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            f = DevFacts{};
+            return false;
+        }
+    }
+    *out = f;
+    return true;
+}
+
 bool decode_plan(const Dims& m, DecPlan* pl) {
     if (m.T < 1 || m.T > kDecMaxT || m.k > kDecMaxK) return false;
-    int dev = 0, optin = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+    DevFacts df;
+    if (!dev_facts(&df)) return false;
+    const int optin = df.optin;
     const int rb_gu = m.d * m.wb / 8, rb_dn = m.f * m.wb / 8;
     if (m.d > 16 * kDecCons) return false;  // the quantiser holds one 16-value piece per consumer thread
     int wbytes = std::max(2 * kDecWarps * rb_gu, kDecWarps * rb_dn);
@@ -41,10 +64,10 @@ bool decode_plan(const Dims& m, DecPlan* pl) {
     // single-token down by output-row ranges: every CTA's rows (whole quads)
     // of one task fit a unit next to the task's codes, and the per-row outputs
     // of all assignments fit the h staging area
-    int sms = 0;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = df.sms;
     const int rr_rows_max = sms > 0 ? (m.d / 4 + sms - 1) / sms * 4 : 1 << 30;
-    q.rowrange = m.T == 1 && m.d % 4 == 0 && q.rd == kDecNQ * kDecWarps && rr_rows_max <= kDecRRMaxRows &&
+    q.rowrange = m.T == 1 && m.k + m.has_shared <= kDecRRMaxTasks && m.d % 4 == 0 &&
+                 q.rd == kDecNQ * kDecWarps && rr_rows_max <= kDecRRMaxRows &&
                  rr_rows_max * rb_dn <= wbytes - m.f && (size_t)m.S * kDecNQ * kDecWarps * 4 <= (size_t)hs;
     q.xs_off = ctl;
     q.hs_off = ctl + xs;
@@ -59,12 +82,12 @@ static cudaError_t go(const Params& p, const DecPlan& pl, const void* x, cudaStr
     auto fn = k_decode<WB, TM, NG, ND, XT>;
     cudaError_t e = allow_smem((const void*)fn, pl.smem_bytes);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kDecThreads, pl.smem_bytes);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+    DevFacts df;
+    if (!dev_facts(&df)) return cudaErrorInvalidDevice;
+    const int sms = df.sms;
+    // one CTA per SM must fit (checked once per kernel, device and size: the
+    // occupancy query costs microseconds of host time per call)
+    if (blocks_per_sm((const void*)fn, pl.smem_bytes, kDecThreads) < 1) return cudaErrorCooperativeLaunchTooLarge;
     const XT* xp = static_cast<const XT*>(x);
     void* args[] = {(void*)&p, (void*)&pl, (void*)&xp};
     return cudaLaunchCooperativeKernel((const void*)fn, dim3(sms), dim3(kDecThreads), args, pl.smem_bytes, s);

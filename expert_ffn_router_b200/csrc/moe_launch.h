@@ -18,7 +18,9 @@ struct ExpertTiling {
 ExpertTiling expert_tiling(int d, int f, int wb);
 
 // Persistent-grid size for a kernel: SMs x resident CTAs (cached per kernel).
-int persistent_grid(const void* func, size_t smem);
+int persistent_grid(const void* func, size_t smem, int threads = kThreads);
+// Resident CTAs per SM (0 if the configuration does not fit), cached.
+int blocks_per_sm(const void* func, size_t smem, int threads);
 // Raise the dynamic shared-memory limit of a kernel once (cached).
 cudaError_t allow_smem(const void* func, size_t smem);
 
