@@ -359,16 +359,18 @@ def gpu_arm(args, wl):
             k_alg = statistics.mean(u * gu_bytes_e for u in uniq)
         achieved = k_alg / k_avg_s / 1e9
         traffic = None
-        try:
+        try:  # ncu DRAM bytes of this kernel and workload, if taken on the current sources
             with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
-                tr = json.load(fh)
+                recs = json.load(fh).get("records", [])
             import importlib.util
             spec = importlib.util.spec_from_file_location("_moe_build", os.path.join(ROOT, "expert_ffn_router_b200",
                                                                                      "build.py"))
             B = importlib.util.module_from_spec(spec)
             spec.loader.exec_module(B)
-            if tr.get("source_hash") == B.source_hash() and tr.get("workload") == wl.name and tr.get("kernel") == kname:
-                traffic = tr.get("bytes_per_launch")
+            h = B.source_hash()
+            for tr in recs:
+                if tr.get("source_hash") == h and tr.get("workload") == wl.name and tr.get("kernel") == kname:
+                    traffic = tr.get("bytes_per_launch")
         except Exception:
             traffic = None
         value = world * K * T / (max_ms / 1e3)
