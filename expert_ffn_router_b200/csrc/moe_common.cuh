@@ -593,6 +593,20 @@ __device__ __forceinline__ int quant_code(float v, float s) {
     return max(-127, min(127, q));
 }
 
+// The same codes without a division per value.  r = quant_recip(s) is the
+// correctly rounded 1/s; q = fl(v r) is within 1.5 * 2^-23 * |v / s| <= 2.3e-5
+// of the IEEE quotient fl(v / s) for |v / s| <= 128 (two roundings of 2^-24
+// each against one), so unless q lies within 1e-3 of a half-integer both round
+// to the same integer; those rare values, and any |q| > 128 (or an infinite
+// r from a denormal s), take the exact quotient.
+__device__ __forceinline__ float quant_recip(float s) { return __fdiv_rn(1.0f, s); }
+__device__ __forceinline__ int quant_code_r(float v, float s, float r) {
+    const float q = __fmul_rn(v, r);
+    const float aq = fabsf(q);
+    if (!(aq <= 128.0f) || fabsf(aq - floorf(aq) - 0.5f) < 1e-3f) return quant_code(v, s);
+    return max(-127, min(127, __float2int_rn(q)));
+}
+
 template <typename XT>
 __device__ __forceinline__ float load_x(const XT* x, size_t i);
 template <>

@@ -628,12 +628,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         }
         m = cons_max(m, C.redf);
         const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+        const float rs = quant_recip(s);
         int cs = 0;
         if (pc < d / 16) {
             unsigned wds[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-                const int code = m == 0.0f ? 0 : quant_code(v[q], s);
+                const int code = m == 0.0f ? 0 : quant_code_r(v[q], s, rs);
                 cs += code;
                 wds[q >> 2] |= ((unsigned)code & 0xFFu) << (8 * (q & 3));
             }
@@ -908,6 +909,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 const int a = min(max(C.ttok[ti][0], 0), p.a_cap - 1);
                 const float m = __uint_as_float(__ldcg(amax_cur + a));
                 const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+                const float rh = quant_recip(sh);
                 int cs = 0;
                 if (ctid < f / 16) {
                     const int pc = ctid;
@@ -919,7 +921,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                         const float hs4[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            const int code = m == 0.0f ? 0 : quant_code(hs4[q], sh);
+                            const int code = m == 0.0f ? 0 : quant_code_r(hs4[q], sh, rh);
                             cs += code;
                             wds[q4] |= ((unsigned)code & 0xFFu) << (8 * q);
                         }
@@ -1014,6 +1016,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 const int a = C.ttok[ti][i];
                 const float m = __uint_as_float(__ldcg(amax_cur + a));
                 const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+                const float rh = quant_recip(sh);
                 const float* hrow = p.ws.h + (size_t)a * f;
                 uint4* hst = reinterpret_cast<uint4*>(hsg) + (size_t)i * NSUB * nch_dn;
                 int cs = 0;
@@ -1025,7 +1028,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                         const float hs4[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            const int code = m == 0.0f ? 0 : quant_code(hs4[q], sh);
+                            const int code = m == 0.0f ? 0 : quant_code_r(hs4[q], sh, rh);
                             cs += code;
                             wds[q4] |= ((unsigned)code & 0xFFu) << (8 * q);
                         }

@@ -142,14 +142,15 @@ __global__ void __launch_bounds__(kThreads) k_gate_up(const Params p) {
                 const int a = s_asg[t];
                 const float m = __uint_as_float(__ldcg(p.ws.amax + a));
                 const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+                const float rh = quant_recip(sh);
                 const float* hrow = p.ws.h + (size_t)a * f;
                 int8_t* qrow = p.ws.hq + (size_t)a * f;
                 for (int c = tid * 4; c < f; c += kThreads * 4) {
                     const float4 hv = __ldcg(reinterpret_cast<const float4*>(hrow + c));
                     char4 q = make_char4(0, 0, 0, 0);
                     if (m != 0.0f)
-                        q = make_char4((signed char)quant_code(hv.x, sh), (signed char)quant_code(hv.y, sh),
-                                       (signed char)quant_code(hv.z, sh), (signed char)quant_code(hv.w, sh));
+                        q = make_char4((signed char)quant_code_r(hv.x, sh, rh), (signed char)quant_code_r(hv.y, sh, rh),
+                                       (signed char)quant_code_r(hv.z, sh, rh), (signed char)quant_code_r(hv.w, sh, rh));
                     *reinterpret_cast<char4*>(qrow + c) = q;
                     if (DBG && p.dbg_hq) *reinterpret_cast<char4*>(p.dbg_hq + (size_t)a * f + c) = q;
                 }

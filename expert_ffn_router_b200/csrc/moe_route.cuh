@@ -18,16 +18,17 @@ __device__ void quantize_token(const XT* x, int d, int8_t* xq, float* sx, int32_
     for (int c = threadIdx.x; c < d; c += kThreads) m = fmaxf(m, fabsf(load_x(x, c)));
     m = block_max(m, redf);
     const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+    const float r = quant_recip(s);
     int cs = 0;
     // d is a multiple of 32: each thread writes 4 codes at a time
     for (int c = threadIdx.x * 4; c < d; c += kThreads * 4) {
         float4 v = load_x4(x, c);
         int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
         if (m != 0.0f) {
-            q0 = quant_code(v.x, s);
-            q1 = quant_code(v.y, s);
-            q2 = quant_code(v.z, s);
-            q3 = quant_code(v.w, s);
+            q0 = quant_code_r(v.x, s, r);
+            q1 = quant_code_r(v.y, s, r);
+            q2 = quant_code_r(v.z, s, r);
+            q3 = quant_code_r(v.w, s, r);
         }
         cs += q0 + q1 + q2 + q3;
         *reinterpret_cast<char4*>(xq + c) = make_char4((signed char)q0, (signed char)q1, (signed char)q2,

@@ -445,6 +445,7 @@ __global__ void __launch_bounds__(kThreads) k_tc_requant(const Params p) {
         const int a = live ? __ldg(p.ws.asg + task.y + j) : 0;
         const float m = live ? __uint_as_float(__ldcg(p.ws.amax + a)) : 0.0f;
         const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+        const float rh = quant_recip(sh);
         const float* hrow = p.ws.h + (size_t)a * f;
         uint8_t* out = p.ws.hb + (size_t)task.w * kpad;
         int cs = 0;
@@ -457,9 +458,10 @@ __global__ void __launch_bounds__(kThreads) k_tc_requant(const Params p) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float4 hv = __ldcg(hp + i);
-                    wv[i] = (uint32_t)(quant_code(hv.x, sh) & 0xFF) | ((uint32_t)(quant_code(hv.y, sh) & 0xFF) << 8) |
-                            ((uint32_t)(quant_code(hv.z, sh) & 0xFF) << 16) |
-                            ((uint32_t)(quant_code(hv.w, sh) & 0xFF) << 24);
+                    wv[i] = (uint32_t)(quant_code_r(hv.x, sh, rh) & 0xFF) |
+                            ((uint32_t)(quant_code_r(hv.y, sh, rh) & 0xFF) << 8) |
+                            ((uint32_t)(quant_code_r(hv.z, sh, rh) & 0xFF) << 16) |
+                            ((uint32_t)(quant_code_r(hv.w, sh, rh) & 0xFF) << 24);
                 }
                 v = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
