@@ -204,7 +204,7 @@ static moe_status check_ws(const moe_config* c, int T, void* ws, size_t ws_bytes
 template <int TM, typename XT>
 static cudaError_t route_small_nv(Params& p, const XT* x, int do_quant, int bucket, cudaStream_t s) {
     const int E = p.m.E;
-    const size_t smem = std::max((size_t)2 * kWarps * E * 4, (size_t)(5 * E + kWarps + kBucketStage) * 4);
+    const size_t smem = std::max((size_t)2 * kWarps * E * 4, (size_t)bucket_smem_ints(E) * 4);
     const int nv = p.m.d / 4;
     const int per = (nv + kThreads - 1) / kThreads;
     const int grid = (E + 1) / 2;
@@ -248,12 +248,18 @@ static cudaError_t launch_router(Params& p, const XT* x, int do_quant, int bucke
     p.ksplit = ks;
     k_router_tiled<XT><<<dim3((E + 63) / 64, (T + 63) / 64, ks), kThreads, 0, s>>>(p, x);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (E <= 256) {  // register top-k; its last CTA buckets
+        const size_t smem_b = bucket ? (size_t)bucket_smem_ints(E) * 4 : 0;
+        if ((e = allow_smem((const void*)k_topk_small, smem_b)) != cudaSuccess) return e;
+        k_topk_small<<<(T + kWarps - 1) / kWarps, kThreads, smem_b, s>>>(p, bucket);
+        return cudaGetLastError();
+    }
     const size_t smem_topk = (size_t)2 * kWarps * E * 4;
     if ((e = allow_smem((const void*)k_topk, smem_topk)) != cudaSuccess) return e;
     k_topk<<<(T + kWarps - 1) / kWarps, kThreads, smem_topk, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (bucket) {
-        const size_t smem_b = (size_t)(5 * E + kWarps + kBucketStage) * 4;
+        const size_t smem_b = (size_t)bucket_smem_ints(E) * 4;
         if ((e = allow_smem((const void*)k_bucket, smem_b)) != cudaSuccess) return e;
         k_bucket<<<1, kThreads, smem_b, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -516,7 +522,7 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         if (e == cudaSuccess) e = launch_combine(q, s);
         if (e == cudaSuccess) e = mark(3);
         if (opts) {
-            opts->n_launches = (T <= 8 ? 1 : 4) + 5;
+            opts->n_launches = (T <= 8 ? 1 : cfg->n_experts <= 256 ? 3 : 4) + 5;
             opts->path_ran = MOE_PATH_TC;
         }
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (tensor cores)");
@@ -528,7 +534,7 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     if (e == cudaSuccess) e = launch_down(p, tl, false, s);
     if (e == cudaSuccess) e = mark(3);
     if (opts) {
-        opts->n_launches = (T <= 8 ? 1 : 4) + 2;
+        opts->n_launches = (T <= 8 ? 1 : cfg->n_experts <= 256 ? 3 : 4) + 2;
         opts->path_ran = MOE_PATH_MULTI;
     }
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer");

@@ -587,6 +587,12 @@ __device__ __forceinline__ int dot_chunk(const uint4 w, const uint4* xs, int nch
 template <int WB>
 __device__ __forceinline__ constexpr int code_offset() { return WB == 4 ? 8 : 2; }
 
+// Order-preserving map of a float to an unsigned key (larger float, larger key).
+__device__ __forceinline__ unsigned float_key(float v) {
+    const unsigned b = __float_as_uint(v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // Quantiser rule of the layer (fp32, IEEE division, round half to even).
 __device__ __forceinline__ int quant_code(float v, float s) {
     int q = __float2int_rn(__fdiv_rn(v, s));

@@ -228,11 +228,6 @@ __device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float
 // NG / ND: 16-byte weight chunks per lane of a gate/up row / a down row when
 // the row is exactly 32 * NG (32 * ND) chunks (fully unrolled, weights loaded
 // up front); 0 = any shape (runtime loop).
-// Order-preserving map of a float to an unsigned key (larger float, larger key).
-__device__ __forceinline__ unsigned float_key(float v) {
-    const unsigned b = __float_as_uint(v);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
 
 // Top-k of one token by one warp for E <= 256: lane l holds experts l + 32 i
 // in registers; each round takes the largest selection score (lowest index on

@@ -123,8 +123,13 @@ static __device__ void topk_token(const Params& p, int t, float* s_sm, float* se
 // counts and zero the per-call counters of the expert kernels.  For
 // tensor-core tasks (p.tc) task.w is the task's first row in the padded
 // operand buffers (the sum of tc_npad over the tasks before it).
-// smem: 5 * E + kWarps + kBucketStage ints.
-constexpr int kBucketStage = 1024;  // routing indices staged per pass of the placement
+// The routing indices pass through shared memory kBucketStage at a time; the
+// stable placement of a stage is split over the warps (each warp a contiguous
+// slice, its per-expert start found by a scan over the warps' histograms).
+// smem: bucket_smem_ints(E) ints.
+constexpr int kBucketStage = 4096;
+__host__ __device__ constexpr int bucket_smem_ints(int E) { return 5 * E + kWarps + kWarps * E + kBucketStage; }
+
 static __device__ void bucket_cta(const Params& p, int* smem) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = p.m.E, k = p.m.k, T = p.m.T, S = p.m.S, CH = p.CH;
@@ -135,19 +140,40 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     int* off0 = smem + 3 * E;
     int* prow = smem + 4 * E;
     int* red = smem + 5 * E;
-    int* stage = red + kWarps;
+    int* hist = red + kWarps;      // [kWarps][E]
+    int* stage = hist + kWarps * E;  // [kBucketStage]
     WsHeader* hdr = p.ws.hdr;
+    // one stage of routing indices into shared memory, four loads in flight per thread
+    auto load_stage = [&](int base, int nb) {
+        for (int i0 = 0; i0 < nb; i0 += 4 * kThreads) {
+            int v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + tid + u * kThreads;
+                v[u] = i < nb ? __ldcg(p.ws.idx + base + i) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + tid + u * kThreads;
+                if (i < nb) {
+                    if (v[u] < 0 || v[u] >= E) {
+                        set_status(hdr, MOE_EDEVICE, base + i);
+                        v[u] = 0;
+                    }
+                    stage[i] = v[u];
+                }
+            }
+        }
+    };
     for (int e = tid; e < E; e += kThreads) cnt[e] = 0;
     __syncthreads();
-    for (int a = tid; a < A; a += kThreads) {
-        int e = __ldcg(p.ws.idx + a);
-        if (e < 0 || e >= E) {
-            set_status(hdr, MOE_EDEVICE, a);
-            e = 0;
-        }
-        atomicAdd(&cnt[e], 1);
+    for (int base = 0; base < A; base += kBucketStage) {
+        const int nb = min(kBucketStage, A - base);
+        load_stage(base, nb);
+        __syncthreads();
+        for (int i = tid; i < nb; i += kThreads) atomicAdd(&cnt[stage[i]], 1);
+        __syncthreads();
     }
-    __syncthreads();
     for (int e = tid; e < E; e += kThreads) {
         off[e] = cnt[e];
         tb[e] = (cnt[e] + CH - 1) / CH;
@@ -162,25 +188,43 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
     const int asg_base = p.m.has_shared ? T : 0;
     const int n_sh_tasks = p.m.has_shared ? (T + CH - 1) / CH : 0;
     const int sh_rows = p.m.has_shared ? (T / CH) * tc_npad(CH) + (T % CH ? tc_npad(T % CH) : 0) : 0;
-    // stable placement by one warp, the indices staged through shared memory
+    // stable placement: warp w takes the contiguous slice [w * per, (w + 1) * per) of a stage
     for (int base = 0; base < A; base += kBucketStage) {
         const int nb = min(kBucketStage, A - base);
-        for (int i = tid; i < nb; i += kThreads) {
-            const int e = __ldcg(p.ws.idx + base + i);
-            stage[i] = (e < 0 || e >= E) ? 0 : e;
+        if (A > kBucketStage) {  // the stage from the counting pass was overwritten
+            load_stage(base, nb);
+        }
+        for (int i = tid; i < kWarps * E; i += kThreads) hist[i] = 0;
+        __syncthreads();
+        const int per = (nb + 32 * kWarps - 1) / (32 * kWarps) * 32;
+        const int lo = warp * per, hi = min(nb, lo + per);
+        for (int b = lo; b < hi; b += 32) {  // per-warp histogram of the slice
+            const int e = b + lane < hi ? stage[b + lane] : E;
+            const unsigned peers = __match_any_sync(kFull, e);
+            if (b + lane < hi && (peers & lanemask_lt()) == 0) hist[warp * E + e] += __popc(peers);
+            __syncwarp();
         }
         __syncthreads();
-        if (warp == 0) {
-            for (int b = 0; b < nb; b += 32) {
-                const int a = base + b + lane;
-                const int e = b + lane < nb ? stage[b + lane] : E;
-                const unsigned peers = __match_any_sync(kFull, e);
-                const int rank = __popc(peers & lanemask_lt());
-                if (b + lane < nb) p.ws.asg[asg_base + off[e] + rank] = (a / k) * S + (a % k);
-                __syncwarp();
-                if (b + lane < nb && rank == 0) off[e] += __popc(peers);
-                __syncwarp();
+        for (int e = tid; e < E; e += kThreads) {  // each warp's first position per expert, in warp order
+            int run = off[e];
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const int h = hist[w * E + e];
+                hist[w * E + e] = run;
+                run += h;
             }
+            off[e] = run;
+        }
+        __syncthreads();
+        for (int b = lo; b < hi; b += 32) {
+            const int a = base + b + lane;
+            const int e = b + lane < hi ? stage[b + lane] : E;
+            const unsigned peers = __match_any_sync(kFull, e);
+            const int rank = __popc(peers & lanemask_lt());
+            if (b + lane < hi) p.ws.asg[asg_base + hist[warp * E + e] + rank] = (a / k) * S + (a % k);
+            __syncwarp();
+            if (b + lane < hi && rank == 0) hist[warp * E + e] += __popc(peers);
+            __syncwarp();
         }
         __syncthreads();
     }
@@ -211,7 +255,7 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
 // 2b+1 for every token (each thread a slice of d, weights streamed once); CTAs
 // b < T also quantise token b.  The last CTA to finish runs the top-k of every
 // token (one warp per token) and, if `bucket`, the bucketing.
-// Dynamic smem: max(2 * kWarps * E floats, 5 * E + kWarps + kBucketStage ints).
+// Dynamic smem: max(2 * kWarps * E floats, bucket_smem_ints(E) ints).
 template <int TM, int NV, typename XT>
 __global__ void __launch_bounds__(kThreads) k_route_small(const Params p, const XT* __restrict__ x,
                                                           int do_quant, int bucket) {
@@ -300,8 +344,12 @@ __global__ void __launch_bounds__(kThreads) k_route_small(const Params p, const 
 // 64 x 64 tile, 32-column k-step, 4 x 4 outputs per thread.
 template <typename XT>
 __global__ void __launch_bounds__(kThreads) k_router_tiled(const Params p, const XT* __restrict__ x) {
-    __shared__ float xs[32][64 + 4];
-    __shared__ float wsm[32][64 + 4];
+    // 64 tokens x 64 experts per CTA over a slice of d (blockIdx.z), 32
+    // columns per step; the next step's tiles are loaded into registers while
+    // the current step's FMAs run (two shared buffers).  Each thread owns a
+    // 4 x 4 block of outputs; sums run in ascending column order per slice.
+    __shared__ __align__(16) float xs[2][32][64 + 4];
+    __shared__ __align__(16) float wsm[2][32][64 + 4];
     const int tid = threadIdx.x;
     const int d = p.m.d, E = p.m.E, T = p.m.T;
     const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
@@ -310,32 +358,52 @@ __global__ void __launch_bounds__(kThreads) k_router_tiled(const Params p, const
     const int kb = blockIdx.z * per, ke = min(ksteps, kb + per);
     const int ty = tid / 16, tx = tid % 16;
     float acc[4][4] = {};
-    for (int ks = kb; ks < ke; ++ks) {
+    float4 xr[2], wr[2];  // this thread's share of one step's tiles: rows r = i / 8, columns (i % 8) * 4
+    auto load = [&](int ks) {
         const int c0 = ks * 32;
-        // 64 rows x 32 columns of x and of W_r: 8 floats per thread each
-        for (int i = tid; i < 64 * 8; i += kThreads) {
-            const int r = i / 8, c4 = (i % 8) * 4;
-            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = xv;
-            if (t0 + r < T) xv = load_x4(x, (size_t)(t0 + r) * d + c0 + c4);
-            if (e0 + r < E) wv = __ldg(reinterpret_cast<const float4*>(p.w_router + (size_t)(e0 + r) * d + c0 + c4));
-            xs[c4 + 0][r] = xv.x; xs[c4 + 1][r] = xv.y; xs[c4 + 2][r] = xv.z; xs[c4 + 3][r] = xv.w;
-            wsm[c4 + 0][r] = wv.x; wsm[c4 + 1][r] = wv.y; wsm[c4 + 2][r] = wv.z; wsm[c4 + 3][r] = wv.w;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = tid + u * kThreads, r = i / 8, c4 = (i % 8) * 4;
+            xr[u] = t0 + r < T ? load_x4(x, (size_t)(t0 + r) * d + c0 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            wr[u] = e0 + r < E ? __ldg(reinterpret_cast<const float4*>(p.w_router + (size_t)(e0 + r) * d + c0 + c4))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        __syncthreads();
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = tid + u * kThreads, r = i / 8, c4 = (i % 8) * 4;
+            xs[buf][c4 + 0][r] = xr[u].x;
+            xs[buf][c4 + 1][r] = xr[u].y;
+            xs[buf][c4 + 2][r] = xr[u].z;
+            xs[buf][c4 + 3][r] = xr[u].w;
+            wsm[buf][c4 + 0][r] = wr[u].x;
+            wsm[buf][c4 + 1][r] = wr[u].y;
+            wsm[buf][c4 + 2][r] = wr[u].z;
+            wsm[buf][c4 + 3][r] = wr[u].w;
+        }
+    };
+    int buf = 0;
+    if (kb < ke) {
+        load(kb);
+        store(0);
+    }
+    __syncthreads();
+    for (int ks = kb; ks < ke; ++ks) {
+        if (ks + 1 < ke) load(ks + 1);  // in flight during the FMAs below
 #pragma unroll 8
         for (int c = 0; c < 32; ++c) {
-            float a[4], b[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a[i] = xs[c][ty * 4 + i];
-                b[i] = wsm[c][tx * 4 + i];
-            }
+            const float4 av = *reinterpret_cast<const float4*>(&xs[buf][c][ty * 4]);
+            const float4 bv = *reinterpret_cast<const float4*>(&wsm[buf][c][tx * 4]);
+            const float a[4] = {av.x, av.y, av.z, av.w}, b[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
         }
+        if (ks + 1 < ke) store(buf ^ 1);
         __syncthreads();
+        buf ^= 1;
     }
     float* dst = p.ws.logits + (size_t)blockIdx.z * T * E;
 #pragma unroll
@@ -358,7 +426,95 @@ __global__ void __launch_bounds__(kThreads) k_topk(const Params p) {
     if (t < p.m.T) topk_token(p, t, dsm + warp * 2 * p.m.E, dsm + warp * 2 * p.m.E + p.m.E);
 }
 
-// Bucketing alone (one CTA).  Dynamic smem (5 * E + kWarps + kBucketStage) ints.
+// Top-k of many tokens for E <= 256: one warp per token, lane l holding
+// experts l + 32 i in registers.  The logits are the ksplit partial planes
+// added in plane order (as topk_token adds them), every plane's loads in
+// flight together; each of the k rounds takes the largest selection value
+// (lowest index on ties) with two warp reductions.  Same rule and arithmetic
+// as topk_token.  With `bucket`, the last CTA to finish runs the bucketing.
+// Dynamic smem: bucket_smem_ints(E) ints if `bucket`.
+__global__ void __launch_bounds__(kThreads) k_topk_small(const Params p, int bucket) {
+    extern __shared__ int bsm[];
+    __shared__ int s_last;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = p.m.E, k = p.m.k, T = p.m.T;
+    const int t = blockIdx.x * kWarps + warp;
+    if (t < T) {
+        float lg[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lg[i] = lane + 32 * i < E ? __ldcg(p.ws.logits + (size_t)t * E + lane + 32 * i) : 0.0f;
+        for (int ks = 1; ks < p.ksplit; ++ks) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                v[i] = lane + 32 * i < E ? __ldcg(p.ws.logits + ((size_t)ks * T + t) * E + lane + 32 * i) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) lg[i] += v[i];
+        }
+        float sv[8];
+        unsigned key[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            sv[i] = 0.0f;
+            key[i] = 0u;  // below every real key
+            if (e < E) {
+                sv[i] = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-lg[i])));
+                key[i] = float_key(__fadd_rn(sv[i], __ldg(p.bias + e)));
+            }
+        }
+        float ssum = 0.0f, my_s = 0.0f;
+        int my_e = 0;
+        for (int j = 0; j < k; ++j) {
+            unsigned best = 0u;
+            int bi = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (key[i] > best) {  // ascending index within the lane: strict keeps the lower one
+                    best = key[i];
+                    bi = i;
+                }
+            const unsigned mx = __reduce_max_sync(kFull, best);
+            const int e_win = __reduce_min_sync(kFull, best == mx ? lane + 32 * bi : 0x7fffffff);
+            const int owner = e_win & 31, slot = e_win >> 5;
+            float s_mine = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i == slot) s_mine = sv[i];
+            const float sj = __shfl_sync(kFull, s_mine, owner);
+            if (lane == owner) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (i == slot) key[i] = 0u;
+            }
+            if (lane == j) {
+                my_e = e_win;
+                my_s = sj;
+            }
+            ssum = __fadd_rn(ssum, sj);
+        }
+        if (lane < k) {
+            const float w = __fmul_rn(__fdiv_rn(my_s, ssum), p.routed_scale);
+            p.ws.idx[(size_t)t * k + lane] = my_e;
+            p.ws.w[(size_t)t * k + lane] = w;
+            if (p.idx_out) p.idx_out[(size_t)t * k + lane] = my_e;
+            if (p.w_out) p.w_out[(size_t)t * k + lane] = w;
+        }
+    }
+    if (!bucket) return;
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        s_last = atomicAdd(&p.ws.hdr->route_ctr, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (tid == 0) p.ws.hdr->route_ctr = 0u;
+    bucket_cta(p, bsm);
+}
+
+// Bucketing alone (one CTA).  Dynamic smem bucket_smem_ints(E) ints.
 __global__ void __launch_bounds__(kThreads) k_bucket(const Params p) {
     extern __shared__ int ism[];
     bucket_cta(p, ism);
