@@ -190,7 +190,7 @@ def reference_arm(args, wl):
 # ---------------------------------------------------------------------------
 TRACE_NAMES = {0: "start", 1: "quantised", 2: "router_done", 3: "shared_gate_up_done", 4: "grid_barrier",
                5: "routing_done", 6: "routed_gate_up_done", 7: "first_down_staged", 8: "down_done",
-               9: "cons_wait_full_total", 10: "prod_wait_empty_total",
+               9: "cons_wait_full_total", 10: "prod_wait_empty_total", 11: "topk_done",
                12: "prod_pre_routing_issued", 13: "prod_routing_received", 14: "prod_all_issued",
                15: "prod_drained"}
 

@@ -9,23 +9,26 @@
 // on an mbarrier per slot).  The consumers work through the same unit
 // sequence, the two consumer groups taking alternate units (4 warps per
 // scheduler to hide the dot products' latencies):
-//   1. router units: logits of this CTA's experts (from x as given), turned
+//   1. the router bias into shared memory;
+//   2. quantise the T tokens (every CTA, into its own shared memory) while
+//      the first rows are on their way;
+//   3. router units: logits of this CTA's experts (from x as given), turned
 //      at once into (selection value, score) pairs -> workspace; arrive at
 //      the one grid barrier;
-//   2. quantise the T tokens (every CTA, into its own shared memory) and run
-//      the shared expert's gate/up units (need no routing) while the
-//      barrier fills;
-//   3. after the barrier every CTA reads all pairs and derives the same
-//      top-k routing and the same expert task list (no second barrier);
-//   4. routed gate/up units; each warp counts the rows it finished per task
-//      and, once at the end of the phase, publishes the counts (one release
-//      fence, then fire-and-forget adds on per-task counters);
-//   5r. single token: one CTA per task requantises the task's h once (after
+//   4. after the barrier every CTA reads all pairs and derives the same
+//      top-k routing and the same expert task list (no second barrier), so
+//      the producer can issue routed rows at once;
+//   5. gate/up units: the shared expert's (their rows were copied before the
+//      routing was known), then the routed ones; each warp counts the rows
+//      it finished per task and, once at the end of the phase, publishes the
+//      counts (one release fence, then fire-and-forget adds on per-task
+//      counters);
+//   6r. single token: one CTA per task requantises the task's h once (after
 //      the task's counter shows every gate/up row) into int8 codes in the
 //      dot layout and publishes them; every CTA then owns a contiguous range
 //      of output rows, streams those rows of every task's down matrix
 //      together with the task's codes, and combines its rows locally;
-//   5. otherwise: down units (waiting, bounded, until their task's counter
+//   6. otherwise: down units (waiting, bounded, until their task's counter
 //      shows every gate/up row) requantise and stage the task's h; at the end
 //      each CTA signs its row blocks off and the CTA bringing a row block's
 //      last task combines it.
@@ -309,6 +312,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         fence_mbar_init();
         C.epoch = __ldcg(&hdr->epoch);
         for (int g = 0; g < kDecGroups; ++g) C.hq_task[g] = -1;
+        if (HS) {  // the shared task (task 0): every token, known before any routing
+            C.tasks[0] = make_int4(E, T, 0, 0);
+            for (int t = 0; t < T; ++t) C.ttok[0][t] = t * S + k;
+        }
     }
     __syncthreads();  // the only CTA-wide barrier: producer and consumers part here
     const uint32_t epoch = C.epoch;
@@ -380,18 +387,33 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             }
             advance();
         }
-        for (int i = 0; i < n_sh_units; ++i) issue_gu(E, c + i * G);
-        DEC_TRACE(12);
-        mbar_wait_bounded(&C.route_ready, 0, hdr, 110);
-        DEC_TRACE(13);
-        const int n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
-        {
-            const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
-            const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
-            int ti = HS + (int)(lo / pl.nu_gu), j = (int)(lo % pl.nu_gu);
-            for (long long g = lo; g < hi; ++g) {
-                issue_gu(C.tasks[ti].x, j);
-                if (++j == pl.nu_gu) {
+        // gate/up rows: the shared expert's units c, c + G, ... first, then,
+        // once the routing is known, this CTA's share of the routed units.
+        // One call site for both (the routed copies are issued by code that
+        // is already in the instruction cache, not by a cold second copy).
+        int n_tasks = HS;
+#pragma unroll 1
+        for (int ph = 0; ph < 2; ++ph) {
+            long long n_units = n_sh_units;
+            int ti = 0, j = c, jstep = G, jwrap = 0x7fffffff, sh_blob = E;
+            if (ph == 1) {
+                DEC_TRACE(12);
+                mbar_wait_bounded(&C.route_ready, 0, hdr, 110);
+                DEC_TRACE(13);
+                n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
+                const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
+                const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
+                n_units = hi - lo;
+                ti = HS + (int)(lo / pl.nu_gu);
+                j = (int)(lo % pl.nu_gu);
+                jstep = 1;
+                jwrap = pl.nu_gu;
+                sh_blob = -1;
+            }
+            for (long long g = 0; g < n_units; ++g) {
+                issue_gu(sh_blob >= 0 ? sh_blob : C.tasks[ti].x, j);
+                j += jstep;
+                if (j == jwrap) {
                     j = 0;
                     ++ti;
                 }
@@ -531,7 +553,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     const bool mine_even = grp == 0;
     auto mine = [&]() { return ((u & 1) == 0) == mine_even; };
 
-    // ---- 2. router units ----
+    // ---- 2. quantise the T tokens into the permuted staging layout (while
+    //         the router rows are on their way) ----
+    for (int t = 0; t < T; ++t) {
+        const XT* xt = x + (size_t)t * d;
+        float v[16];
+        float m = 0.0f;
+        const int pc = ctid;  // d / 16 <= kDecCons pieces of 16 values
+        if (pc < d / 16) {
+            load16(xt, (size_t)pc * 16, v);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) m = fmaxf(m, fabsf(v[q]));
+        }
+        m = cons_max(m, C.redf);
+        const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
+        const float rs = quant_recip(s);
+        int cs = 0;
+        if (pc < d / 16) {
+            unsigned wds[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int code = m == 0.0f ? 0 : quant_code_r(v[q], s, rs);
+                cs += code;
+                wds[q >> 2] |= ((unsigned)code & 0xFFu) << (8 * (q & 3));
+            }
+            xs[(size_t)t * NSUB * nch_gu + (pc % NSUB) * nch_gu + pc / NSUB] =
+                permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
+        }
+        cs = cons_sum_int(cs, C.redi);
+        if (ctid == 0) {
+            C.sx[t] = s;
+            C.xcs[t] = cs;
+        }
+    }
+    named_sync(kDecBar, kDecCons);
+    if (ctid == 0) DEC_TRACE(1);
+    for (int i = c * kDecCons + ctid; i < p.a_cap; i += G * kDecCons) amax_nxt[i] = 0u;
+    for (int i = c * kDecCons + ctid; i < kDecMaxTasks; i += G * kDecCons) rows_nxt[i] = 0u;
+
+    // ---- 3. router units ----
     for (int ru = 0; ru < n_router_units; ++ru, next_unit()) {
         if (!mine()) continue;
         const int rows = min(pl.rr, n_my_router - ru * pl.rr);
@@ -608,42 +668,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             st_release_u32(&hdr->b1_gen, epoch + 1);
         }
     }
-
-    // ---- 2b. quantise the T tokens into the permuted staging layout (while the
-    //          grid barrier fills) ----
-    for (int t = 0; t < T; ++t) {
-        const XT* xt = x + (size_t)t * d;
-        float v[16];
-        float m = 0.0f;
-        const int pc = ctid;  // d / 16 <= kDecCons pieces of 16 values
-        if (pc < d / 16) {
-            load16(xt, (size_t)pc * 16, v);
-#pragma unroll
-            for (int q = 0; q < 16; ++q) m = fmaxf(m, fabsf(v[q]));
-        }
-        m = cons_max(m, C.redf);
-        const float s = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
-        const float rs = quant_recip(s);
-        int cs = 0;
-        if (pc < d / 16) {
-            unsigned wds[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int code = m == 0.0f ? 0 : quant_code_r(v[q], s, rs);
-                cs += code;
-                wds[q >> 2] |= ((unsigned)code & 0xFFu) << (8 * (q & 3));
-            }
-            xs[(size_t)t * NSUB * nch_gu + (pc % NSUB) * nch_gu + pc / NSUB] =
-                permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
-        }
-        cs = cons_sum_int(cs, C.redi);
-        if (ctid == 0) {
-            C.sx[t] = s;
-            C.xcs[t] = cs;
-        }
-    }
-    named_sync(kDecBar, kDecCons);
-    if (ctid == 0) DEC_TRACE(1);
 
     // ---- per-warp gate/up bookkeeping ----
     // Rows finished per task are counted in registers and published once, at
@@ -784,113 +808,118 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         ++cur_cnt;
     };
 
-    // ---- 3. shared-expert gate/up units (no routing needed) ----
-    if (n_sh_units > 0) {  // the shared task's description, known before routing
-        if (ctid < T) C.ttok[0][ctid] = ctid * S + k;
-        if (ctid == 0) C.tasks[0] = make_int4(E, T, 0, 0);
-        named_sync(kDecBar, kDecCons);
-    }
-    for (int i = 0; i < n_sh_units; ++i, next_unit())
-        if (mine()) gu_unit(0, c + i * G);
-
-    if (ctid == 0) DEC_TRACE(3);
-    // ---- 4. grid barrier, then every CTA derives the routing ----
-    if (ctid == 0) flag_wait_bounded(&hdr->b1_gen, epoch + 1, hdr, 300);
-    named_sync(kDecBar, kDecCons);
-    if (ctid == 0) DEC_TRACE(4);
-    if (c == 0 && ctid == 0) hdr->epoch = epoch + 1;
-    for (int i = c * kDecCons + ctid; i < p.a_cap; i += G * kDecCons) amax_nxt[i] = 0u;
-    for (int i = c * kDecCons + ctid; i < kDecMaxTasks; i += G * kDecCons) rows_nxt[i] = 0u;
-    if (warp < T) {
-        int my_e;
-        float my_w;
-        if (E <= kDecBiasCache) {
-            topk_warp_small(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale,
-                            my_e, my_w);
-        } else {
-            float* scr = reinterpret_cast<float*>(hsb) + (size_t)warp * 2 * E;
-            topk_warp(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale, scr,
-                      scr + E, my_e, my_w);
-        }
-        if (lane < k) {
-            C.idx[warp][lane] = my_e;
-            C.w[warp][lane] = my_w;
-            if (c == 0) {
-                p.ws.idx[warp * k + lane] = my_e;
-                p.ws.w[warp * k + lane] = my_w;
-                if (p.idx_out) p.idx_out[warp * k + lane] = my_e;
-                if (p.w_out) p.w_out[warp * k + lane] = my_w;
+    // ---- 4-5. gate/up units, with the grid barrier and the routing
+    //      between them.  The group that does not own this CTA's last router
+    //      unit runs the first shared-expert unit before the routing (its rows
+    //      were copied with the router rows; running gu_unit once there brings
+    //      its code into the instruction cache while HBM is otherwise idle);
+    //      the remaining shared units and the routed units follow the routing.
+    //      One call site of gu_unit for every unit: a second inlined copy would
+    //      start cold, with its fetches on the critical path after the routing.
+    int n_tasks = HS;
+    const int n_sh_first = min(n_sh_units, 1);
+#pragma unroll 1
+    for (int ph = 0; ph < 3; ++ph) {
+        long long n_units = n_sh_first;
+        int ti = 0, j = c, jstep = G, jwrap = 0x7fffffff;  // shared: units c, c + G, ... of task 0
+        if (ph == 1) {
+            // ---- 4. grid barrier, then every CTA derives the routing ----
+            if (ctid == 0) flag_wait_bounded(&hdr->b1_gen, epoch + 1, hdr, 300);
+            named_sync(kDecBar, kDecCons);
+            if (ctid == 0) DEC_TRACE(4);
+            if (c == 0 && ctid == 0) hdr->epoch = epoch + 1;
+            if (warp < T) {
+                int my_e;
+                float my_w;
+                if (E <= kDecBiasCache) {
+                    topk_warp_small(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale,
+                                    my_e, my_w);
+                } else {
+                    float* scr = reinterpret_cast<float*>(hsb) + (size_t)warp * 2 * E;
+                    topk_warp(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale, scr,
+                              scr + E, my_e, my_w);
+                }
+                if (lane < k) {
+                    C.idx[warp][lane] = my_e;
+                    C.w[warp][lane] = my_w;
+                    if (c == 0) {
+                        p.ws.idx[warp * k + lane] = my_e;
+                        p.ws.w[warp * k + lane] = my_w;
+                        if (p.idx_out) p.idx_out[warp * k + lane] = my_e;
+                        if (p.w_out) p.w_out[warp * k + lane] = my_w;
+                    }
+                }
             }
-        }
-    }
-    named_sync(kDecBar, kDecCons);
-    // bucket: sort the T*k assignments by (expert, token, slot); one task per expert
-    const int A = T * k;
-    if (T == 1) {  // one token: the k experts, each a task with that token, by ascending expert
-        if (warp == 0) {
-            const int e = lane < k ? C.idx[0][lane] : 0x7fffffff;
-            int rank = 0;
-            for (int j = 0; j < k; ++j) rank += __shfl_sync(kFull, e, j) < e;
-            if (lane < k) {
-                C.ttok[HS + rank][0] = lane;  // assignment id: token 0, slot lane
-                C.tasks[HS + rank] = make_int4(e, 1, 0, 0);
+            named_sync(kDecBar, kDecCons);
+            if (ctid == 0) DEC_TRACE(11);
+            // bucket: sort the T*k assignments by (expert, token, slot); one task per expert
+            const int A = T * k;
+            if (T == 1) {  // one token: the k experts, each a task with that token, by ascending expert
+                if (warp == 0) {
+                    const int e = lane < k ? C.idx[0][lane] : 0x7fffffff;
+                    int rank = 0;
+                    for (int jj = 0; jj < k; ++jj) rank += __shfl_sync(kFull, e, jj) < e;
+                    if (lane < k) {
+                        C.ttok[HS + rank][0] = lane;  // assignment id: token 0, slot lane
+                        C.tasks[HS + rank] = make_int4(e, 1, 0, 0);
+                    }
+                    if (lane == 0) C.n_tasks = HS + k;
+                }
+            } else if (ctid < A) {
+                const int ea = C.idx[ctid / k][ctid % k];
+                int pos = 0, a2 = 0;
+                for (int t2 = 0; t2 < T; ++t2)
+                    for (int j2 = 0; j2 < k; ++j2, ++a2) {
+                        const int e2 = C.idx[t2][j2];
+                        pos += (e2 < ea) || (e2 == ea && a2 < ctid);
+                    }
+                C.sorted[pos] = ctid;
+                C.sorted_e[pos] = ea;
             }
-            if (HS && lane == 0) {
-                C.ttok[0][0] = k;
-                C.tasks[0] = make_int4(E, 1, 0, 0);
+            named_sync(kDecBar, kDecCons);
+            if (T > 1 && ctid < A) {
+                const int a = C.sorted[ctid];
+                const int ea = C.sorted_e[ctid];
+                int tq = -1, rank = 0, n = 0;
+                for (int q = 0; q <= ctid; ++q) {
+                    const int eq = C.sorted_e[q];
+                    tq += eq != (q == 0 ? -1 : C.sorted_e[q - 1]);
+                    rank += (eq == ea) && q < ctid;
+                }
+                for (int q = 0; q < A; ++q) n += C.sorted_e[q] == ea;
+                C.ttok[HS + tq][rank] = (a / k) * S + (a % k);
+                if (rank == 0) C.tasks[HS + tq] = make_int4(ea, n, 0, 0);
+                if (ctid == A - 1) C.n_tasks = HS + tq + 1;
             }
-            if (lane == 0) C.n_tasks = HS + k;
-        }
-    } else if (ctid < A) {
-        const int ea = C.idx[ctid / k][ctid % k];
-        int pos = 0, a2 = 0;
-        for (int t2 = 0; t2 < T; ++t2)
-            for (int j2 = 0; j2 < k; ++j2, ++a2) {
-                const int e2 = C.idx[t2][j2];
-                pos += (e2 < ea) || (e2 == ea && a2 < ctid);
+            named_sync(kDecBar, kDecCons);
+            if (ctid == 0) {
+                mbar_arrive(&C.route_ready);  // the producer may issue routed rows
+                DEC_TRACE(5);
             }
-        C.sorted[pos] = ctid;
-        C.sorted_e[pos] = ea;
-    }
-    if (T > 1 && HS && ctid < T) C.ttok[0][ctid] = ctid * S + k;
-    if (T > 1 && HS && ctid == 0) C.tasks[0] = make_int4(E, T, 0, 0);
-    named_sync(kDecBar, kDecCons);
-    if (T > 1 && ctid < A) {
-        const int a = C.sorted[ctid];
-        const int ea = C.sorted_e[ctid];
-        int ti = -1, rank = 0, n = 0;
-        for (int q = 0; q <= ctid; ++q) {
-            const int eq = C.sorted_e[q];
-            ti += eq != (q == 0 ? -1 : C.sorted_e[q - 1]);
-            rank += (eq == ea) && q < ctid;
+            n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
+            n_units = n_sh_units - n_sh_first;
+            j = c + n_sh_first * G;
+        } else if (ph == 2) {
+            if (ctid == 0) DEC_TRACE(3);
+            const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
+            const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
+            n_units = hi - lo;
+            ti = HS + (int)(lo / pl.nu_gu);
+            j = (int)(lo % pl.nu_gu);
+            jstep = 1;
+            jwrap = pl.nu_gu;
         }
-        for (int q = 0; q < A; ++q) n += C.sorted_e[q] == ea;
-        C.ttok[HS + ti][rank] = (a / k) * S + (a % k);
-        if (rank == 0) C.tasks[HS + ti] = make_int4(ea, n, 0, 0);
-        if (ctid == A - 1) C.n_tasks = HS + ti + 1;
-    }
-    named_sync(kDecBar, kDecCons);
-    if (ctid == 0) {
-        mbar_arrive(&C.route_ready);  // the producer may issue routed rows
-        DEC_TRACE(5);
-    }
-    const int n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
-
-    // ---- 5. routed gate/up units ----
-    {
-        const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
-        const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
-        int ti = HS + (int)(lo / pl.nu_gu), j = (int)(lo % pl.nu_gu);
-        for (long long g = lo; g < hi; ++g, next_unit()) {
+        for (long long g = 0; g < n_units; ++g, next_unit()) {
             if (mine()) gu_unit(ti, j);
-            if (++j == pl.nu_gu) {
+            j += jstep;
+            if (j == jwrap) {
                 j = 0;
                 ++ti;
             }
         }
-        flush_gu();
-        publish(0);
     }
+    flush_gu();
+    publish(0);
     if (ctid == 0) DEC_TRACE(6);
 
     // ---- 6r. single token: row-range down with a local combine ----
