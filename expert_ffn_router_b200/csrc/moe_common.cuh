@@ -235,6 +235,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_u32(bar)) : "memory");
 }
+// Non-blocking test of a phase (try_wait may suspend the thread for a while
+// before it reports "not yet", which delays whatever else a polling loop does).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -267,6 +278,9 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 }
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 // Fire-and-forget add (no value returned to the thread).
 __device__ __forceinline__ void red_add_u32(uint32_t* p, uint32_t v) {
@@ -606,10 +620,15 @@ __device__ __forceinline__ int quant_code(float v, float s) {
 // to the same integer; those rare values, and any |q| > 128 (or an infinite
 // r from a denormal s), take the exact quotient.
 __device__ __forceinline__ float quant_recip(float s) { return __fdiv_rn(1.0f, s); }
+// The exact quotient out of line: taken for well under 1% of values, it keeps
+// the division's instructions out of every unrolled copy of the fast path
+// (code that a kernel runs once per call is fetched cold, from HBM, while the
+// weight streams saturate it).
+static __device__ __noinline__ int quant_code_slow(float v, float s) { return quant_code(v, s); }
 __device__ __forceinline__ int quant_code_r(float v, float s, float r) {
     const float q = __fmul_rn(v, r);
     const float aq = fabsf(q);
-    if (!(aq <= 128.0f) || fabsf(aq - floorf(aq) - 0.5f) < 1e-3f) return quant_code(v, s);
+    if (!(aq <= 128.0f) || fabsf(aq - floorf(aq) - 0.5f) < 1e-3f) return quant_code_slow(v, s);
     return max(-127, min(127, __float2int_rn(q)));
 }
 

@@ -56,6 +56,7 @@ constexpr int kDecBiasCache = 256;  // experts whose bias the kernel keeps in sh
 constexpr int kDecBar = 1;  // named barrier of all consumer warps; 2 + g: group g
 constexpr int kDecNQ = 6;   // down rows per warp per unit of the unrolled shapes (rd = 48)
 constexpr int kDecXr = 8;   // router float4 inputs per thread for one token (d <= 8 * 4 * 256)
+constexpr int kDecTraceSlots = 32;  // phase stamps per CTA (moe_layer_opts.trace)
 
 struct DecPlan {
     int slot_bytes, nslot;
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     const int nch_gu = rb_gu / 16, nch_dn = rb_dn / 16;
     const int nslot = pl.nslot, slot_bytes = pl.slot_bytes;
     WsHeader* hdr = p.ws.hdr;
-    unsigned long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * 16 : nullptr;
+    unsigned long long* trace = p.trace ? p.trace + (size_t)blockIdx.x * kDecTraceSlots : nullptr;
 #define DEC_TRACE(i)                                   \
     do {                                               \
         if (trace) trace[i] = global_timer_ns();       \
@@ -434,6 +435,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     mbar_arrive_expect_tx(&C.codes[next_code], (uint32_t)f + 16);
                     bulk_g2s(dsts[next_code] + pl.wbytes - f, p.ws.hq + (size_t)a * f, (uint32_t)f, &C.codes[next_code]);
                     bulk_g2s(dsts[next_code] + pl.wbytes + kDecRRMetaOff, p.ws.hmeta + a, 16, &C.codes[next_code]);
+                    if (next_code == 0) DEC_TRACE(18);
+                    DEC_TRACE(19);
                     ++next_code;
                 }
             };
@@ -441,7 +444,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             for (int ti = 0; ti < n_rr; ++ti) {
                 if (pr > 0) {  // wait for the slot, servicing published codes meanwhile
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&C.empty[ps], (pr - 1) & 1)) {
+                    while (!mbar_test_wait(&C.empty[ps], (pr - 1) & 1)) {
                         issue_codes(ti);
                         if (global_timer_ns() - t0 > kWaitLimitNs) {
                             set_status(hdr, MOE_ETIMEOUT, 131);
@@ -656,16 +659,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         }
         named_sync(2 + grp, kDecGrp);
     }
-    // arrive at the grid barrier (logits of this CTA published)
-    __threadfence();
+    // arrive at the grid barrier (logits of this CTA published).  One fence
+    // per CTA and one for the last arrival: a fence costs microseconds once
+    // the weight streams load HBM.
     named_sync(kDecBar, kDecCons);
     if (ctid == 0) {
         DEC_TRACE(2);
+        fence_acq_rel_gpu();  // release: the CTA's logits, ordered by the barrier, before the arrival
         const unsigned ticket = atomicAdd(&hdr->b1_count, 1u);
         if (ticket == (unsigned)G - 1) {
-            hdr->b1_count = 0u;
-            __threadfence();
-            st_release_u32(&hdr->b1_gen, epoch + 1);
+            hdr->b1_count = 0u;  // read again only by the next launch
+            fence_acq_rel_gpu();  // acquire every arrival's logits, release them with the flag
+            st_relaxed_u32(&hdr->b1_gen, epoch + 1);
         }
     }
 
@@ -927,21 +932,31 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         if (rowrange) {
             // requantise the tasks this CTA is designated for (task ti -> CTA ti % G)
             for (int ti = c; ti < n_tasks; ti += G) {
-                if (ctid == 0) flag_wait_bounded(rows_cur + ti, (uint32_t)(pl.nu_gu * kDecWarps), hdr, 410);
+                if (ctid == 0) {
+                    flag_wait_bounded(rows_cur + ti, (uint32_t)(pl.nu_gu * kDecWarps), hdr, 410);
+                    if (ti == c) DEC_TRACE(16);
+                }
+                // thread 0's acquire of the count, passed on by the barrier,
+                // orders the loads below after the other CTAs' h rows and
+                // maxima (their fence precedes their count); no second fence
                 named_sync(kDecBar, kDecCons);
-                __threadfence();  // the other CTAs' h rows and maxima
                 const int a = min(max(C.ttok[ti][0], 0), p.a_cap - 1);
+                const int pc = ctid;
+                const float* hrow = p.ws.h + (size_t)a * f;
+                float4 hv4[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    hv4[q4] = pc < f / 16 ? __ldcg(reinterpret_cast<const float4*>(hrow + pc * 16 + 4 * q4))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
                 const float m = __uint_as_float(__ldcg(amax_cur + a));
                 const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
                 const float rh = quant_recip(sh);
                 int cs = 0;
-                if (ctid < f / 16) {
-                    const int pc = ctid;
-                    const float* hrow = p.ws.h + (size_t)a * f;
+                if (pc < f / 16) {
                     unsigned wds[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
-                        const float4 hv = __ldcg(reinterpret_cast<const float4*>(hrow + pc * 16 + 4 * q4));
+                        const float4 hv = hv4[q4];
                         const float hs4[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -953,11 +968,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     reinterpret_cast<uint4*>(p.ws.hq + (size_t)a * f)[(pc % NSUB) * nch_dn + pc / NSUB] =
                         permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
                 }
-                cs = cons_sum_int(cs, C.redi);  // its barrier orders every thread's codes before thread 0's fence
+                cs = cons_sum_int(cs, C.redi);  // its barrier orders every thread's codes before thread 0's release
                 if (ctid == 0) {
                     p.ws.hmeta[a] = make_int4(__float_as_int(sh), cs, 0, 0);
-                    __threadfence();
-                    st_release_u32(hq_ready + ti, epoch + 1);  // readers fence the async proxy before copying
+                    // one release (cumulative over the barrier) publishes codes
+                    // and record; readers fence the async proxy before copying
+                    st_release_u32(hq_ready + ti, epoch + 1);
+                    if (ti == c) DEC_TRACE(17);
                 }
             }
             if (ctid == 0) DEC_TRACE(7);
@@ -969,6 +986,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 if (!mine()) continue;
                 const uint8_t* slot = wait_full();
                 mbar_wait_bounded(&C.codes[ti], 0, hdr, 420);
+                if (ti == 0 && ctid == 0) DEC_TRACE(20);
                 uint4 hrr[ND][NSUB];
                 const uint4* hq4 = reinterpret_cast<const uint4*>(slot + pl.wbytes - f);
 #pragma unroll
@@ -1003,6 +1021,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 }
             }
             named_sync(kDecBar, kDecCons);  // every y of this CTA's rows is in shared memory
+            if (ctid == 0) DEC_TRACE(21);
             for (int rl = ctid; rl < rr_rows; rl += kDecCons) {
                 float o = 0.0f;
                 for (int jj = 0; jj < k; ++jj) o = fmaf(C.w[0][jj], ys[jj * RRW + rl], o);

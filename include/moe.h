@@ -180,14 +180,19 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *        when T >= tc_min_tokens, else MULTI.
  *  path_ran: set to the path that ran (MOE_PATH_DECODE, _MULTI or _TC).
  *  n_launches: set to the number of kernels the call launched.
- *  trace: optional DEVICE buffer of (number of SMs) x 16 uint64 that the
+ *  trace: optional DEVICE buffer of (number of SMs) x 32 uint64 that the
  *         single-launch decode path fills with per-CTA global-timer stamps
  *         (ns) at its phase boundaries: [0] start, [1] tokens quantised,
  *         [2] router rows done, [3] shared-expert gate/up done, [4] grid
  *         barrier passed, [5] routing derived, [6] routed gate/up done,
- *         [7] first down staging ready, [8] down done; producer: [12] rows
- *         known before routing issued, [13] routing received, [14] all rows
- *         issued, [15] all copies landed.  Untouched entries are left as is. */
+ *         [7] first down staging ready, [8] down done, [11] top-k done;
+ *         totals: [9] consumer wait for data, [10] producer wait for slots;
+ *         producer: [12] rows known before routing issued, [13] routing
+ *         received, [14] all rows issued, [15] all copies landed, [18] first
+ *         and [19] last copy of published codes issued; single-token down:
+ *         [16] the CTA's designated task fully counted, [17] its codes
+ *         published, [20] first down unit's codes landed, [21] last down
+ *         unit done.  Untouched entries are left as is. */
 enum { MOE_PATH_AUTO = 0, MOE_PATH_MULTI = 1, MOE_PATH_DECODE = 2, MOE_PATH_TC = 3 };
 typedef struct {
     void* events[4];
