@@ -301,9 +301,11 @@ def gpu_arm(args, wl):
         torch.cuda.synchronize()
     barrier()
     step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(K)]
-    route_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    gu_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    dn_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(K)]
+    # the single-launch decode path records only events [0] and [3]
+    phased = opts[0].path_ran != M.MOE_PATH_DECODE
+    route_ms = [ev[i][0].elapsed_time(ev[i][1]) if phased else 0.0 for i in range(K)]
+    gu_ms = [ev[i][1].elapsed_time(ev[i][2]) if phased else 0.0 for i in range(K)]
+    dn_ms = [ev[i][2].elapsed_time(ev[i][3]) if phased else 0.0 for i in range(K)]
     total_ms = sum(step_ms)
     assert M.moe_poll_status(ws) == M.MOE_OK
 
