@@ -44,16 +44,42 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments, whitespace runs collapsed; string
+    and character literals are kept as written."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash() -> str:
-    """Hash of every source and header the library is built from (ties a
-    recorded ncu traffic figure to the kernel it was measured on)."""
+    """Hash of the code (comments and layout ignored) of every source and
+    header the library is built from: ties a recorded ncu traffic figure to
+    the kernel it was measured on."""
     import hashlib
     h = hashlib.sha256()
     for p in sorted(_deps()):
         if p.endswith(".py"):
             continue
-        with open(p, "rb") as fh:
-            h.update(os.path.basename(p).encode() + fh.read())
+        with open(p, encoding="utf-8") as fh:
+            h.update(os.path.basename(p).encode() + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

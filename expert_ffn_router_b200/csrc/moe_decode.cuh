@@ -14,15 +14,16 @@
 //      the first rows are on their way;
 //   3. router units: logits of this CTA's experts (from x as given), turned
 //      at once into (selection value, score) pairs -> workspace; arrive at
-//      the one grid barrier;
+//      the one grid barrier; meanwhile the other consumer group runs the
+//      CTA's first shared-expert gate/up unit (its rows were copied with the
+//      router rows);
 //   4. after the barrier every CTA reads all pairs and derives the same
 //      top-k routing and the same expert task list (no second barrier), so
 //      the producer can issue routed rows at once;
-//   5. gate/up units: the shared expert's (their rows were copied before the
-//      routing was known), then the routed ones; each warp counts the rows
-//      it finished per task and, once at the end of the phase, publishes the
-//      counts (one release fence, then fire-and-forget adds on per-task
-//      counters);
+//   5. gate/up units: the remaining shared-expert ones, then the routed ones;
+//      each warp counts the rows it finished per task and, once at the end
+//      of the phase, publishes the counts (one release fence, then
+//      fire-and-forget adds on per-task counters);
 //   6r. single token: one CTA per task requantises the task's h once (after
 //      the task's counter shows every gate/up row) into int8 codes in the
 //      dot layout and publishes them; every CTA then owns a contiguous range
