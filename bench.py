@@ -192,9 +192,8 @@ TRACE_NAMES = {0: "start", 1: "quantised", 2: "router_done", 3: "shared_gate_up_
                5: "routing_done", 6: "routed_gate_up_done", 7: "first_down_staged", 8: "down_done",
                9: "cons_wait_full_total", 10: "prod_wait_empty_total", 11: "topk_done",
                12: "prod_pre_routing_issued", 13: "prod_routing_received", 14: "prod_all_issued",
-               15: "prod_drained", 16: "designated_task_counted", 17: "designated_codes_published",
-               18: "prod_first_codes_issued", 19: "prod_last_codes_issued", 20: "first_down_codes_landed",
-               21: "last_down_unit_done"}
+               15: "prod_drained", 16: "designated_h_row_complete", 17: "designated_codes_written",
+               20: "first_down_codes_seen", 21: "last_down_unit_done"}
 
 
 def write_trace(path, M, cfg, pool, dl, xbuf, out, ws, dev, flush_l2):

@@ -282,6 +282,45 @@ __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
 __device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Morally strong (relaxed, gpu-scope) accesses for values that other CTAs poll
+// without a fence: each reader checks every value it uses against the preset
+// "not written" pattern, so no ordering between values is needed.
+constexpr uint32_t kNotWritten = 0x7fbadbadu;  // a NaN payload that arithmetic never produces
+constexpr uint32_t kCodesNotWritten = 0x80808080u;  // -128 bytes: never a code
+__device__ __forceinline__ void st_relaxed_f32(float* p, float v) {
+    asm volatile("st.relaxed.gpu.global.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+__device__ __forceinline__ float ld_relaxed_f32(const float* p) {
+    float v;
+    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 ld_relaxed_f4(const float* p) {
+    float4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ uint4 ld_relaxed_u4(const void* p) {
+    uint4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_u4(void* p, uint4 v) {
+    asm volatile("st.relaxed.gpu.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+// Nonzero iff some byte of w is 0x80.
+__device__ __forceinline__ uint32_t has_byte_80(uint32_t w) {
+    const uint32_t v = w ^ 0x80808080u;
+    return (v - 0x01010101u) & ~v & 0x80808080u;
+}
 // Fire-and-forget add (no value returned to the thread).
 __device__ __forceinline__ void red_add_u32(uint32_t* p, uint32_t v) {
     asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");

@@ -21,14 +21,17 @@
 //      top-k routing and the same expert task list (no second barrier), so
 //      the producer can issue routed rows at once;
 //   5. gate/up units: the remaining shared-expert ones, then the routed ones;
-//      each warp counts the rows it finished per task and, once at the end
-//      of the phase, publishes the counts (one release fence, then
-//      fire-and-forget adds on per-task counters);
-//   6r. single token: one CTA per task requantises the task's h once (after
-//      the task's counter shows every gate/up row) into int8 codes in the
-//      dot layout and publishes them; every CTA then owns a contiguous range
-//      of output rows, streams those rows of every task's down matrix
-//      together with the task's codes, and combines its rows locally;
+//      with several tokens each warp counts the rows it finished per task
+//      and, once at the end of the phase, publishes the counts (one release
+//      fence, then fire-and-forget adds on per-task counters);
+//   6r. single token: no counts and no fences -- the call's h rows, code
+//      rows and scales are preset to "not written" before the grid barrier;
+//      one CTA per task polls the task's h values until all are written,
+//      requantises them into int8 codes in the dot layout (max |h| from the
+//      values themselves) and writes codes and scale; every CTA owns a
+//      contiguous range of output rows, streams those rows of every task's
+//      down matrix, polls the task's codes and scale straight from global
+//      memory, and combines its rows locally;
 //   6. otherwise: down units (waiting, bounded, until their task's counter
 //      shows every gate/up row) requantise and stage the task's h; at the end
 //      each CTA signs its row blocks off and the CTA bringing a row block's
@@ -69,17 +72,14 @@ struct DecPlan {
     int hs_grp_bytes;  // h staging bytes of one consumer group (T * f)
     int rowrange;      // single-token down by output-row ranges (see step 6r)
 };
-// Row-range down unit (single token): [rows x down row][.. hq codes at
-// wbytes - f][row scales at wbytes][(scale, code sum) record at wbytes + 176].
+// Row-range down unit (single token): [rows x down row][row scales at wbytes].
 constexpr int kDecRRMaxRows = 44;
-constexpr int kDecRRMetaOff = 4 * kDecNQ * kDecWarps - 16;
 
 constexpr int kDecRRMaxTasks = kDecMaxK + 1;  // tasks of a single token (row-range down)
 
 struct DecCtl {
     uint64_t full[kDecMaxSlots];
     uint64_t empty[kDecMaxSlots];
-    uint64_t codes[kDecRRMaxTasks];  // row-range down: task ti's codes landed in its unit's slot
     uint64_t route_ready;
     uint32_t epoch;
     int n_tasks;
@@ -310,7 +310,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             mbar_init(&C.empty[i], kDecWarps);
         }
         mbar_init(&C.route_ready, 1);
-        for (int i = 0; i < kDecRRMaxTasks; ++i) mbar_init(&C.codes[i], 1);
         fence_mbar_init();
         C.epoch = __ldcg(&hdr->epoch);
         for (int g = 0; g < kDecGroups; ++g) C.hq_task[g] = -1;
@@ -328,7 +327,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     // the same for the per-task counts of finished gate/up rows
     uint32_t* rows_cur = p.ws.ready + (epoch & 1) * 1024;
     uint32_t* rows_nxt = p.ws.ready + ((epoch & 1) ^ 1) * 1024;
-    uint32_t* hq_ready = p.ws.ready + 2048;
     // this CTA's output rows in the row-range down: whole quads of rows, so
     // the row scales are whole 16-byte bulk copies
     const int rr_lo = (int)((long long)c * (d / 4) / G) * 4;
@@ -423,62 +421,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         }
         if (rowrange) {
             // one unit per task: this CTA's rows of the task's down matrix and
-            // their scales at once; the task's published codes and (scale,
-            // code sum) record follow into the same slot, counted on
-            // C.codes[ti], as soon as the task's flag is seen -- serviced
-            // while waiting for slots, so the weights never wait for the codes
-            uint8_t* dsts[kDecRRMaxTasks];
-            int next_code = 0;
-            auto issue_codes = [&](int n_units) {  // the codes of every published task in order
-                while (next_code < n_units && ld_acquire_u32(hq_ready + next_code) == epoch + 1) {
-                    fence_proxy_async_all();  // the codes were stored by another CTA's threads
-                    const int a = min(max(C.ttok[next_code][0], 0), p.a_cap - 1);
-                    mbar_arrive_expect_tx(&C.codes[next_code], (uint32_t)f + 16);
-                    bulk_g2s(dsts[next_code] + pl.wbytes - f, p.ws.hq + (size_t)a * f, (uint32_t)f, &C.codes[next_code]);
-                    bulk_g2s(dsts[next_code] + pl.wbytes + kDecRRMetaOff, p.ws.hmeta + a, 16, &C.codes[next_code]);
-                    if (next_code == 0) DEC_TRACE(18);
-                    DEC_TRACE(19);
-                    ++next_code;
-                }
-            };
+            // their scales (the consumers read the task's codes from global
+            // memory themselves, once written)
             const int n_rr = min(n_tasks, kDecRRMaxTasks);
             for (int ti = 0; ti < n_rr; ++ti) {
-                if (pr > 0) {  // wait for the slot, servicing published codes meanwhile
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_test_wait(&C.empty[ps], (pr - 1) & 1)) {
-                        issue_codes(ti);
-                        if (global_timer_ns() - t0 > kWaitLimitNs) {
-                            set_status(hdr, MOE_ETIMEOUT, 131);
-                            break;
-                        }
-                    }
-                }
                 const int blob = min(max(C.tasks[ti].x, 0), n_blobs - 1);
-                uint64_t* bar = &C.full[ps];
                 const uint32_t wb = (uint32_t)rr_rows * rb_dn;
-                mbar_arrive_expect_tx(bar, wb + (uint32_t)rr_rows * 4);
-                uint8_t* dst = ring + (size_t)ps * slot_bytes;
-                dsts[ti] = dst;
+                uint8_t* dst = take(wb + (uint32_t)rr_rows * 4);
                 bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)rr_lo * rb_dn, wb,
-                         bar);
+                         &C.full[ps]);
                 bulk_g2s(dst + pl.wbytes, p.scales + (size_t)blob * p.scale_rows + 2 * f + rr_lo, (uint32_t)rr_rows * 4,
-                         bar);
+                         &C.full[ps]);
                 advance();
-                issue_codes(ti + 1);
             }
-            {  // the codes still unpublished: wait for them in order (bounded)
-                const uint64_t t0 = global_timer_ns();
-                while (next_code < n_rr) {
-                    issue_codes(n_rr);
-                    if (next_code < n_rr && ld_volatile_status(hdr) != 0) break;
-                    if (global_timer_ns() - t0 > kWaitLimitNs) {
-                        set_status(hdr, MOE_ETIMEOUT, 132);
-                        break;
-                    }
-                }
-            }
-            // every code copy issued has landed before the CTA can retire
-            for (int ti = 0; ti < next_code; ++ti) mbar_wait_bounded(&C.codes[ti], 0, hdr, 133);
         } else {
             const long long Nd = (long long)n_tasks * pl.nu_dn;
             const long long lo = c * Nd / G, hi = (c + 1) * Nd / G;
@@ -594,6 +549,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     if (ctid == 0) DEC_TRACE(1);
     for (int i = c * kDecCons + ctid; i < p.a_cap; i += G * kDecCons) amax_nxt[i] = 0u;
     for (int i = c * kDecCons + ctid; i < kDecMaxTasks; i += G * kDecCons) rows_nxt[i] = 0u;
+    if (rowrange) {
+        // single token: the h rows, code rows and scales of the call's S
+        // assignments start as "not written", so that the gate/up -> down
+        // hand-off needs no fence (a fence issued while the weight streams
+        // saturate HBM takes microseconds): the requantiser polls the h values
+        // and the down units poll the codes and scale.  The grid barrier below
+        // orders these stores before every write of this call.
+        const uint4 hn = make_uint4(kNotWritten, kNotWritten, kNotWritten, kNotWritten);
+        const uint4 qn = make_uint4(kCodesNotWritten, kCodesNotWritten, kCodesNotWritten, kCodesNotWritten);
+        for (int i = c * kDecCons + ctid; i < S * f / 4; i += G * kDecCons) reinterpret_cast<uint4*>(p.ws.h)[i] = hn;
+        for (int i = c * kDecCons + ctid; i < S * f / 16; i += G * kDecCons) reinterpret_cast<uint4*>(p.ws.hq)[i] = qn;
+        if (c == G - 1 && ctid < S) reinterpret_cast<uint32_t*>(p.ws.sh)[ctid] = kNotWritten;
+    }
 
     // ---- 3. router units ----
     for (int ru = 0; ru < n_router_units; ++ru, next_unit()) {
@@ -698,7 +666,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         t_sx[i] = 0.0f;
     }
     auto publish = [&](int n_keep) {  // publish all but the newest n_keep pending counts
-        fence_acq_rel_gpu();          // this warp's h stores and maxima before its counts
+        if (n_pend <= n_keep) return;  // (warp-uniform)
+        fence_acq_rel_gpu();           // this warp's h stores and maxima before its counts
         __syncwarp();
         if (lane == 0)
             for (int i = 0; i < n_pend - n_keep; ++i) red_add_u32(rows_cur + pend_task[i], (uint32_t)pend_cnt[i]);
@@ -710,6 +679,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     };
     auto flush_gu = [&]() {  // close the current task: maxima now, the row count later
         if (cur_task < 0 || cur_cnt == 0) return;
+        if (rowrange) {  // single token: the requantiser reads the h values themselves
+            cur_cnt = 0;
+            return;
+        }
 #pragma unroll
         for (int i = 0; i < TM; ++i)
             if (i < cur_n && lane == i) atomicMax(amax_cur + t_asg[i], __float_as_uint(amax[i]));
@@ -805,7 +778,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                         const float g = __fmul_rn((float)Gv, __fmul_rn(sg, t_sx[i]));
                         const float uu = __fmul_rn((float)Uv, __fmul_rn(su, t_sx[i]));
                         const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), uu);
-                        p.ws.h[(size_t)t_asg[i] * f + r] = h;
+                        st_relaxed_f32(p.ws.h + (size_t)t_asg[i] * f + r, h);
                         amax[i] = fmaxf(amax[i], fabsf(h));
                     }
                 }
@@ -931,50 +904,57 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     // ---- 6r. single token: row-range down with a local combine ----
     if constexpr (TM == 1 && ND > 0) {
         if (rowrange) {
-            // requantise the tasks this CTA is designated for (task ti -> CTA ti % G)
+            // requantise the tasks this CTA is designated for (task ti -> CTA
+            // ti % G): poll the task's h values until every one is written,
+            // max |h| over the row, then the codes and the scale, with relaxed
+            // stores that the down units poll in turn (no count, no fence)
             for (int ti = c; ti < n_tasks; ti += G) {
-                if (ctid == 0) {
-                    flag_wait_bounded(rows_cur + ti, (uint32_t)(pl.nu_gu * kDecWarps), hdr, 410);
-                    if (ti == c) DEC_TRACE(16);
-                }
-                // thread 0's acquire of the count, passed on by the barrier,
-                // orders the loads below after the other CTAs' h rows and
-                // maxima (their fence precedes their count); no second fence
-                named_sync(kDecBar, kDecCons);
-                const int a = min(max(C.ttok[ti][0], 0), p.a_cap - 1);
+                const int a = min(max(C.ttok[ti][0], 0), S - 1);
                 const int pc = ctid;
-                const float* hrow = p.ws.h + (size_t)a * f;
                 float4 hv4[4];
+                float m = 0.0f;
+                if (pc < f / 16) {
+                    const float* src = p.ws.h + (size_t)a * f + pc * 16;
+                    const uint64_t t0 = global_timer_ns();
+                    for (;;) {
+                        bool ok = true;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    hv4[q4] = pc < f / 16 ? __ldcg(reinterpret_cast<const float4*>(hrow + pc * 16 + 4 * q4))
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float m = __uint_as_float(__ldcg(amax_cur + a));
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            hv4[q4] = ld_relaxed_f4(src + 4 * q4);
+                            ok = ok && __float_as_uint(hv4[q4].x) != kNotWritten && __float_as_uint(hv4[q4].y) != kNotWritten &&
+                                 __float_as_uint(hv4[q4].z) != kNotWritten && __float_as_uint(hv4[q4].w) != kNotWritten;
+                        }
+                        if (ok) break;
+                        if (global_timer_ns() - t0 > kWaitLimitNs || ld_volatile_status(hdr) != 0) {
+                            set_status(hdr, MOE_ETIMEOUT, 410);
+                            break;
+                        }
+                    }
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        m = fmaxf(fmaxf(fmaxf(m, fabsf(hv4[q4].x)), fmaxf(fabsf(hv4[q4].y), fabsf(hv4[q4].z))),
+                                  fabsf(hv4[q4].w));
+                }
+                m = cons_max(m, C.redf);
+                if (ctid == 0 && ti == c) DEC_TRACE(16);
                 const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
                 const float rh = quant_recip(sh);
-                int cs = 0;
                 if (pc < f / 16) {
                     unsigned wds[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
-                        const float4 hv = hv4[q4];
-                        const float hs4[4] = {hv.x, hv.y, hv.z, hv.w};
+                        const float hs4[4] = {hv4[q4].x, hv4[q4].y, hv4[q4].z, hv4[q4].w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int code = m == 0.0f ? 0 : quant_code_r(hs4[q], sh, rh);
-                            cs += code;
                             wds[q4] |= ((unsigned)code & 0xFFu) << (8 * q);
                         }
                     }
-                    reinterpret_cast<uint4*>(p.ws.hq + (size_t)a * f)[(pc % NSUB) * nch_dn + pc / NSUB] =
-                        permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3]));
+                    st_relaxed_u4(reinterpret_cast<uint4*>(p.ws.hq + (size_t)a * f) + (pc % NSUB) * nch_dn + pc / NSUB,
+                                  permute16<WB>(make_uint4(wds[0], wds[1], wds[2], wds[3])));
                 }
-                cs = cons_sum_int(cs, C.redi);  // its barrier orders every thread's codes before thread 0's release
                 if (ctid == 0) {
-                    p.ws.hmeta[a] = make_int4(__float_as_int(sh), cs, 0, 0);
-                    // one release (cumulative over the barrier) publishes codes
-                    // and record; readers fence the async proxy before copying
-                    st_release_u32(hq_ready + ti, epoch + 1);
+                    st_relaxed_f32(p.ws.sh + a, sh);
                     if (ti == c) DEC_TRACE(17);
                 }
             }
@@ -986,15 +966,44 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             for (int ti = 0; ti < min(n_tasks, kDecRRMaxTasks); ++ti, next_unit()) {
                 if (!mine()) continue;
                 const uint8_t* slot = wait_full();
-                mbar_wait_bounded(&C.codes[ti], 0, hdr, 420);
-                if (ti == 0 && ctid == 0) DEC_TRACE(20);
+                const int a = min(max(C.ttok[ti][0], 0), S - 1);
+                // the task's scale and codes straight from global memory, each
+                // polled until written (the whole code row sits in the warp)
+                float shv = 0.0f;
                 uint4 hrr[ND][NSUB];
-                const uint4* hq4 = reinterpret_cast<const uint4*>(slot + pl.wbytes - f);
+                {
+                    const uint4* hq4 = reinterpret_cast<const uint4*>(p.ws.hq + (size_t)a * f);
+                    const uint64_t t0 = global_timer_ns();
+                    for (;;) {
+                        shv = ld_relaxed_f32(p.ws.sh + a);
+                        uint32_t bad = __float_as_uint(shv) == kNotWritten;
+#pragma unroll
+                        for (int i = 0; i < ND; ++i)
+#pragma unroll
+                            for (int sb = 0; sb < NSUB; ++sb) {
+                                hrr[i][sb] = ld_relaxed_u4(hq4 + sb * nch_dn + lane + 32 * i);
+                                bad |= has_byte_80(hrr[i][sb].x) | has_byte_80(hrr[i][sb].y) | has_byte_80(hrr[i][sb].z) |
+                                       has_byte_80(hrr[i][sb].w);
+                            }
+                        if (!__any_sync(kFull, bad != 0u)) break;
+                        if (global_timer_ns() - t0 > kWaitLimitNs || ld_volatile_status(hdr) != 0) {
+                            set_status(hdr, MOE_ETIMEOUT, 420);
+                            break;
+                        }
+                    }
+                }
+                if (ti == 0 && gtid == 0) DEC_TRACE(20);
+                int csl = 0;  // the code sum, for the offset-binary correction
 #pragma unroll
                 for (int i = 0; i < ND; ++i)
 #pragma unroll
-                    for (int sb = 0; sb < NSUB; ++sb) hrr[i][sb] = hq4[sb * nch_dn + lane + 32 * i];
-                const int4 meta = *reinterpret_cast<const int4*>(slot + pl.wbytes + kDecRRMetaOff);
+                    for (int sb = 0; sb < NSUB; ++sb) {
+                        csl = __dp4a((int)hrr[i][sb].x, 0x01010101, csl);
+                        csl = __dp4a((int)hrr[i][sb].y, 0x01010101, csl);
+                        csl = __dp4a((int)hrr[i][sb].z, 0x01010101, csl);
+                        csl = __dp4a((int)hrr[i][sb].w, 0x01010101, csl);
+                    }
+                const int cs = __reduce_add_sync(kFull, csl);
                 const float* sd = reinterpret_cast<const float*>(slot + pl.wbytes);
                 uint4 wv[kDecNQ][ND];
                 float sdr[kDecNQ];
@@ -1009,14 +1018,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     sdr[q] = ok ? sd[rl] : 0.0f;
                 }
                 release();
-                const float shv = __int_as_float(meta.x);
-                const int a = min(max(C.ttok[ti][0], 0), S - 1);
 #pragma unroll
                 for (int q = 0; q < kDecNQ; ++q) {
                     int a0 = 0, a1 = 0;
 #pragma unroll
                     for (int i = 0; i < ND; ++i) dot_chunk_regs<WB>(wv[q][i], hrr[i], a0, a1);
-                    const int D = __reduce_add_sync(kFull, a0 + a1) - code_offset<WB>() * meta.y;
+                    const int D = __reduce_add_sync(kFull, a0 + a1) - code_offset<WB>() * cs;
                     const int rl = q * kDecWarps + gw;
                     if (lane == 0 && rl < rr_rows) ys[a * RRW + rl] = __fmul_rn((float)D, __fmul_rn(sdr[q], shv));
                 }

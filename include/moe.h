@@ -189,11 +189,11 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *         [7] first down staging ready, [8] down done, [11] top-k done;
  *         totals: [9] consumer wait for data, [10] producer wait for slots;
  *         producer: [12] rows known before routing issued, [13] routing
- *         received, [14] all rows issued, [15] all copies landed, [18] first
- *         and [19] last copy of published codes issued; single-token down:
- *         [16] the CTA's designated task fully counted, [17] its codes
- *         published, [20] first down unit's codes landed, [21] last down
- *         unit done.  Untouched entries are left as is. */
+ *         received, [14] all rows issued, [15] all copies landed; single-token
+ *         down: [16] the CTA's designated task's h row complete (polled),
+ *         [17] its codes and scale written, [20] first down unit's codes
+ *         seen, [21] last down unit done.  Untouched entries are left as
+ *         is. */
 enum { MOE_PATH_AUTO = 0, MOE_PATH_MULTI = 1, MOE_PATH_DECODE = 2, MOE_PATH_TC = 3 };
 typedef struct {
     void* events[4];
