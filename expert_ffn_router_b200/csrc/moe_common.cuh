@@ -39,8 +39,8 @@ struct WsHeader {
 static_assert(sizeof(WsHeader) == 256, "header must stay 256 bytes");
 
 // Decode-kernel control words after the header: [0, 1024) and [1024, 2048)
-// gate/up rows finished per task (the two halves alternate by call parity),
-// [2048, 3072) per-task "requantised h published" flags (epoch valued).
+// gate/up rows finished per task (the two halves alternate by call parity;
+// several-token calls), [2048, 4096) reserved.
 constexpr int kReadyFlags = 4096;
 constexpr size_t kCtrlBytes = sizeof(WsHeader) + kReadyFlags * 4;  // zeroed by moe_workspace_init
 
@@ -64,7 +64,7 @@ struct Ws {
     float* ybuf;       // [T*S][d]   per-assignment down outputs before the combine
     uint32_t* rb_ctr;  // [ceil(d/rb4)] down item arrivals per row block (self-resetting)
     int32_t* hcs;      // [T*S]      sum of the hq codes of each assignment (tensor-core down)
-    int4* hmeta;       // [T*S]      (scale bits, code sum, -, -) of each assignment's hq (decode down)
+    int4* hmeta;       // [T*S]      reserved (no path writes it)
     uint8_t* xb;       // tensor-core operand B of gate/up: per task, activation rows in MMA layout
     uint8_t* hb;       // tensor-core operand B of down: per task, hq rows in MMA layout
     size_t bytes;

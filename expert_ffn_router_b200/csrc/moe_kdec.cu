@@ -62,8 +62,9 @@ bool decode_plan(const Dims& m, DecPlan* pl) {
     q.nslot = std::min(kDecMaxSlots, room / slot) / 2 * 2;
     if (q.nslot < 2) return false;
     // single-token down by output-row ranges: every CTA's rows (whole quads)
-    // of one task fit a unit next to the task's codes, and the per-row outputs
-    // of all assignments fit the h staging area
+    // of one task fit a unit with f bytes to spare (the set of shapes this
+    // path has been measured and tested on), and the per-row outputs of all
+    // assignments fit the h staging area
     const int sms = df.sms;
     const int rr_rows_max = sms > 0 ? (m.d / 4 + sms - 1) / sms * 4 : 1 << 30;
     q.rowrange = m.T == 1 && m.k + m.has_shared <= kDecRRMaxTasks && m.d % 4 == 0 &&
