@@ -49,6 +49,37 @@ def parse():
     return ap.parse_args()
 
 
+def metric_for(wl, workload_id):
+    """The headline metric on its own workload; a labelled variant elsewhere."""
+    return METRIC if workload_id == 1 else f"MoE-layer tokens/s on {wl.name}; expert-weight HBM GB/s"
+
+
+def dtype_for(wl):
+    return "i8*i4->i32" if wl.wbits == 4 else "i8*i2->i32"
+
+
+def rank_token_sets(rank, n_sets):
+    """Seeds of a rank's token stream: every replica draws its own tokens
+    (rank 0's stream is the single-GPU one)."""
+    return [rank * 1000 + s for s in range(n_sets)]
+
+
+def max_over_ranks(ms, world, dist=None, device=None):
+    """The slowest rank's time: every rank calls this (the same collective in
+    the same order on all ranks) and gets the maximum."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, steps, tokens_per_step, max_ms):
+    """Tokens per second of all ranks together over the slowest rank's time."""
+    return world * steps * tokens_per_step / (max_ms / 1e3)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -166,21 +197,24 @@ def reference_arm(args, wl):
     if rank != 0:
         return
     K, Wm = args.steps, args.warmup
-    run = oracle_decode_timer(wl, 0, list(range(min(100, K + Wm))))
+    # a bounded sample per step: the whole token for decode, at most 4 tokens
+    # of a batched workload (the oracle's per-token cost does not depend on T)
+    per = min(wl.T, 4)
+    run = oracle_decode_timer(wl, 0, list(range(min(100, K + Wm))), max_tokens=per)
     for i in range(Wm):
         run(i)
     t0 = time.perf_counter()
     for i in range(K):
         run(Wm + i)
     el = time.perf_counter() - t0
-    v = K * wl.T / el
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": K,
-            "warmup": Wm, "ms_per_step": 1e3 * el / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "i8*i4->i32", "data": "synthetic",
+    v = K * per / el
+    line = {"impl": "reference", "metric": metric_for(wl, args.workload), "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": K, "warmup": Wm, "ms_per_step": 1e3 * el / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype_for(wl), "data": "synthetic",
             "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "f": wl.f, "experts": wl.n_experts,
                        "shared": wl.has_shared, "top_k": wl.top_k, "wbits": wl.wbits},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
-                             "sample": f"{K} timed tokens of {wl.name}, full layer per token"},
+                             "sample": f"{K} timed steps of {per} token(s) of {wl.name}, full layer"},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -250,7 +284,7 @@ def gpu_arm(args, wl):
     pool = M.make_pool(dl.pool_w, dl.pool_s)
     n_sets = wl.n_token_sets
     # every rank draws its own token stream
-    toks = torch.stack([W.tokens(wl, 0, rank * 1000 + s) for s in range(n_sets)]).to(dev)  # [n_sets][T][d]
+    toks = torch.stack([W.tokens(wl, 0, s) for s in rank_token_sets(rank, n_sets)]).to(dev)  # [n_sets][T][d]
     xbuf = torch.empty(T, wl.d, dtype=toks.dtype, device=dev)
     out = torch.empty(T, wl.d, device=dev)
     idx = torch.empty(T, wl.top_k, dtype=torch.int32, device=dev)
@@ -315,10 +349,7 @@ def gpu_arm(args, wl):
     dn_bytes_e = wl.d * wl.f * wl.wbits // 8 + wl.d * 4
     exp_bytes = sum(u * (gu_bytes_e + dn_bytes_e) for u in uniq)
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(total_ms, world, dist, dev)
 
     e2e = None
     if not args.no_e2e:
@@ -338,10 +369,8 @@ def gpu_arm(args, wl):
             e_e[i].record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = torch.tensor([sum(e_s[i].elapsed_time(e_e[i]) for i in range(K))], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * K * T / (float(e2e_ms.item()) / 1e3), "unit": "tokens/s",
+        e2e_ms = max_over_ranks(sum(e_s[i].elapsed_time(e_e[i]) for i in range(K)), world, dist, dev)
+        e2e = {"value": whole_job_rate(world, K, T, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": T * wl.d * toks.element_size(), "d2h_bytes_per_step": T * wl.d * 4,
                "api": "expert_ffn_router_b200.moe_layer (libmoe.so moe_layer), pinned host buffers"}
 
@@ -376,13 +405,13 @@ def gpu_arm(args, wl):
                     traffic = tr.get("bytes_per_launch")
         except Exception:
             traffic = None
-        value = world * K * T / (max_ms / 1e3)
+        value = whole_job_rate(world, K, T, max_ms)
         exp_gbs = exp_bytes / (total_ms / 1e3) / 1e9
         line = {
-            "metric": METRIC if args.workload == 1 else f"MoE-layer tokens/s on {wl.name}; expert-weight HBM GB/s",
+            "metric": metric_for(wl, args.workload),
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "i8*i4->i32" if wl.wbits == 4 else "i8*i2->i32", "data": "synthetic",
+            "dtype": dtype_for(wl), "data": "synthetic",
             "config": {"workload": wl.name, "T": T, "d": wl.d, "f": wl.f, "experts": wl.n_experts,
                        "shared": wl.has_shared, "top_k": wl.top_k, "wbits": wl.wbits,
                        "pool_gb": wl.pool_bytes / 1e9, "token_sets": n_sets,
