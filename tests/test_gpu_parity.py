@@ -217,6 +217,37 @@ def test_layer_decode_full_size():
     print("decode rel L2 per call:", errs)
 
 
+def test_layer_decode_repeats_bit_identical():
+    """The single-token decode layer called 300 times on 6 tokens in turn,
+    with an L2 flush before every other call: each token's output repeats bit
+    for bit.  Its gate/up -> down hand-off has no fence (readers poll values
+    preset to "not written"), so a stale or torn read would show here as a
+    differing output (the outputs' agreement with the oracle is
+    test_layer_decode_full_size's)."""
+    wl = W.workload(1)
+    dl = W.device_layer(wl, 0, 0)
+    cfg = cfg_of(wl)
+    pool = M.make_pool(dl.pool_w, dl.pool_s)
+    ws = M.workspace(cfg, 1)
+    out = torch.empty(1, wl.d, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    toks = [to_dev(x_host(wl, s)) for s in range(6)]
+    refs, bad = {}, 0
+    for it in range(300):
+        i = it % 6
+        if it % 2 == 0:
+            flush.fill_(it & 0xFF)
+        M.moe_layer(cfg, pool, dl.w_router, dl.bias, toks[i], out, ws)
+        o = out.clone()
+        if i in refs:
+            bad += int(not torch.equal(o, refs[i]))
+        else:
+            refs[i] = o
+    torch.cuda.synchronize()
+    assert_ok(ws)
+    assert bad == 0
+
+
 def test_layer_decode_int2_full_size():
     wl = W.workload(4)
     L = W.layer(wl, 0, 0)
