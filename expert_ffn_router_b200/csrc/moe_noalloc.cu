@@ -10,7 +10,6 @@
 // every GPU that loads the library holds until the process exits.
 #include <cuda_runtime.h>
 
-#include <mutex>
 #include <string>
 
 #include "moe.h"
@@ -30,26 +29,21 @@ static_assert(sizeof(WsHeader) + (size_t)kStaticMaxT * kStaticMaxE * 4 + 2 * (si
 
 static __device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
 
-// Device address of g_route_scratch on each device, looked up once per device
-// (with that device current).  In host code the array's name stands for a
-// host-side shadow, never for the device memory itself.
-static std::mutex g_scratch_mu;
-static void* g_scratch_ptr[128];
-
+// Device address of g_route_scratch on the current device.  In host code the
+// array's name stands for a host-side shadow, never for the device memory
+// itself, so the address is looked up with the device current.  The lookup is
+// repeated on every call (it costs well under a microsecond of host time): an
+// address kept from an earlier call would be stale after the caller resets the
+// device, which unloads and reloads the library's module.
 static moe_status scratch_for_current_device(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(MOE_ECUDA, std::string("moe_route_static: cudaGetDevice: ") + cudaGetErrorString(e));
-    if (dev < 0 || dev >= 128) return fail(MOE_EINVAL, "moe_route_static: device index out of range");
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_route_scratch);
-        if (e != cudaSuccess || !ptr)
-            return fail(MOE_ECUDA, std::string("moe_route_static: cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-        g_scratch_ptr[dev] = ptr;
-    }
-    *out = g_scratch_ptr[dev];
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_route_scratch);
+    if (e != cudaSuccess || !ptr)
+        return fail(MOE_ECUDA, std::string("moe_route_static: cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    *out = ptr;
     return MOE_OK;
 }
 

@@ -16,7 +16,9 @@ import pytest
 import torch
 
 import expert_ffn_router_b200 as M
+import oracle as O
 import workloads as W
+from parity_utils import routing_mismatches
 
 FAKE = 1 << 20
 
@@ -33,10 +35,16 @@ def test_static_router_rejects_requests_beyond_its_limit():
     assert M.lib.moe_route_static(ctypes.byref(c), FAKE, 1, 0, FAKE, FAKE, FAKE, FAKE, None) == M.MOE_OK
 
 
+WIDE = W.workload(0).replace(name="tiny_E1024_k32", n_experts=1024, top_k=32, T=8)
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("which,T", [(0, 5), (1, 1), (1, 8)])
+@pytest.mark.parametrize("which,T", [(0, 5), (1, 1), (1, 8), ("wide", 8)])
 def test_static_router_matches_workspace_router(which, T):
-    wl = W.workload(which)
+    """The E = 1024, k = 32 case is the largest the static limits allow: the
+    router's logits fill the array's largest region, and the top-k uses all
+    32 lanes of its warp; it is also checked against the CPU oracle."""
+    wl = WIDE if which == "wide" else W.workload(which)
     cfg = cfg_of(wl)
     L = W.layer(wl, 0, 0)
     wr, bias = L.w_router.cuda(), L.bias.cuda()
@@ -52,3 +60,8 @@ def test_static_router_matches_workspace_router(which, T):
         torch.cuda.synchronize()
         np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx.cpu().numpy())
         np.testing.assert_allclose(w.cpu().numpy(), ref_w.cpu().numpy(), rtol=2e-6, atol=1e-7)
+        if which == "wide":
+            o_idx, _, _, _, o_sel = O.route(x.float(), L.w_router, L.bias, wl.top_k, wl.routed_scale,
+                                            want_scores=True)
+            _, bad = routing_mismatches(idx.cpu().numpy(), o_idx, o_sel)
+            assert bad == []
