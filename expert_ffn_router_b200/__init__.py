@@ -17,7 +17,9 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe.so")
+# MOE_LIBRARY=bounds loads the bounds-checked build (every index the kernels
+# read from data range-checked into the status word), for tests
+LIB_PATH = os.path.join(_PKG, "libmoe_bounds.so" if os.environ.get("MOE_LIBRARY") == "bounds" else "libmoe.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "moe.h")
 
 MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_ENOSPACE, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE = 0, -1, -2, -3, -4, -5, -6
@@ -51,7 +53,8 @@ class MoeConfig(ctypes.Structure):
 
 class MoeLayerOpts(ctypes.Structure):
     _fields_ = [("events", ctypes.c_void_p * 4), ("path", ctypes.c_int32), ("n_launches", ctypes.c_int32),
-                ("trace", ctypes.c_void_p), ("path_ran", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("trace", ctypes.c_void_p), ("path_ran", ctypes.c_int32),
+                ("wait_limit_us", ctypes.c_int32), ("test_skip_h", ctypes.c_int32)]
 
 
 class MoePool(ctypes.Structure):

@@ -1,4 +1,4 @@
-"""Build libmoe.so (sm_100a) in-tree.
+"""Build libmoe.so (sm_100a) in-tree, and its bounds-checked twin.
 
     python expert_ffn_router_b200/build.py [--force] [--verbose]
 
@@ -7,8 +7,11 @@
 Each .cu translation unit under csrc/ is compiled in parallel with
 ``nvcc -gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` and the objects
 are linked into expert_ffn_router_b200/libmoe.so (static CUDA runtime, no
-torch dependency).  The build is skipped when the library is newer than every
-source and header.
+torch dependency).  libmoe_bounds.so is the same library compiled with
+MOE_BOUNDS: every index the kernels read from data is range-checked and a
+violation is recorded as MOE_EDEVICE in the workspace's status word (the
+package loads it instead when MOE_LIBRARY=bounds).  A build is skipped when
+its library is newer than every source and header.
 """
 import concurrent.futures as cf
 import glob
@@ -22,6 +25,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
+LIB_BOUNDS = os.path.join(PKG, "libmoe_bounds.so")
 BUILD = os.path.join(PKG, "_build")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -83,16 +87,16 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+def _compile(src: str, verbose: bool, extra, tag: str) -> str:
+    obj = os.path.join(BUILD, os.path.basename(src) + tag + ".o")
+    cmd = [nvcc()] + NVCC_FLAGS + list(extra) + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{r.stderr}")
@@ -101,18 +105,26 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def _build_one(lib: str, extra, tag: str, force: bool, verbose: bool) -> str:
+    if not force and up_to_date(lib):
+        return lib
     os.makedirs(BUILD, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=max(1, min(len(sources()), os.cpu_count() or 1))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), sources()))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose, extra, tag), sources()))
+    tmp = lib + ".tmp"
     cmd = [nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp] + objs + ["-cudart", "static"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False, bounds: bool = True) -> str:
+    """Build libmoe.so (and libmoe_bounds.so unless bounds=False); returns libmoe.so's path."""
+    _build_one(LIB, [], "", force, verbose)
+    if bounds:
+        _build_one(LIB_BOUNDS, ["-DMOE_BOUNDS"], ".bounds", force, verbose)
     return LIB
 
 

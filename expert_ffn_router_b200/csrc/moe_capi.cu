@@ -158,6 +158,8 @@ static int tc_nt_max(int T) { return tc_npad(std::min(T, kTcNT)); }
 static Params base_params(const moe_config* c, const Dims& m, void* ws, size_t ws_bytes, bool tc = false) {
     Params p{};
     p.m = m;
+    p.wait_ns = kWaitLimitNs;
+    p.skip_h_task = -1;
     p.routed_scale = c->routed_scale;
     p.blob_bytes = 3ll * c->d * c->f * c->wbits / 8;
     p.scale_rows = 2 * c->f + c->d;
@@ -457,6 +459,8 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     if (opts) {
         opts->n_launches = 0;
         opts->path_ran = MOE_PATH_AUTO;
+        if (opts->wait_limit_us < 0 || opts->test_skip_h < 0)
+            return fail(MOE_EINVAL, "opts->wait_limit_us and opts->test_skip_h must be >= 0");
     }
     if (T == 0) return MOE_OK;
     MOE_TRY(check_ptr(pool->w, "pool->w"));
@@ -479,6 +483,8 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     p.idx_out = topk_idx_out;
     p.w_out = topk_w_out;
     p.trace = opts ? static_cast<unsigned long long*>(opts->trace) : nullptr;
+    if (opts && opts->wait_limit_us > 0) p.wait_ns = (unsigned long long)opts->wait_limit_us * 1000ull;
+    if (opts && opts->test_skip_h > 0) p.skip_h_task = opts->test_skip_h - 1;
     cudaStream_t s = (cudaStream_t)stream;
     const ExpertTiling tl = expert_tiling(cfg->d, cfg->f, cfg->wbits);
     auto mark = [&](int i) -> cudaError_t {
@@ -490,11 +496,15 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         return fail(MOE_EINVAL, "opts->path must be MOE_PATH_AUTO, MOE_PATH_MULTI, MOE_PATH_DECODE or MOE_PATH_TC");
     DecPlan pl{};
     const bool dec_ok = (path == MOE_PATH_AUTO || path == MOE_PATH_DECODE) && decode_plan(m, &pl);
+    // the h-skip hook acts only where the hand-off polls values (one token,
+    // row-range down); elsewhere it would give wrong output instead of a timeout
+    if (!(dec_ok && pl.rowrange)) p.skip_h_task = -1;
     if (path == MOE_PATH_DECODE && !dec_ok) return fail(MOE_EINVAL, "shape does not fit the single-launch decode path");
     if (path == MOE_PATH_TC && !tc_shape_ok(m)) return fail(MOE_EINVAL, "shape does not fit the tensor-core path");
     cudaError_t e = mark(0);
     if (dec_ok) {
-        if (e == cudaSuccess) e = launch_decode(p, pl, x, dtype == MOE_BF16, s);
+        if (e == cudaSuccess)
+            e = launch_decode(p, pl, x, dtype == MOE_BF16, s);
         if (e == cudaSuccess) e = mark(3);  // [1] and [2] fall inside the one kernel: not recorded
         if (opts) {
             opts->n_launches = 1;

@@ -39,9 +39,9 @@ struct WsHeader {
 static_assert(sizeof(WsHeader) == 256, "header must stay 256 bytes");
 
 // Decode-kernel control words after the header: [0, 1024) and [1024, 2048)
-// gate/up rows finished per task (the two halves alternate by call parity;
-// several-token calls), [2048, 4096) reserved.
-constexpr int kReadyFlags = 4096;
+// gate/up rows finished per task of the several-token kernel (the two halves
+// alternate by call parity).
+constexpr int kReadyFlags = 2048;
 constexpr size_t kCtrlBytes = sizeof(WsHeader) + kReadyFlags * 4;  // zeroed by moe_workspace_init
 
 struct Ws {
@@ -64,7 +64,6 @@ struct Ws {
     float* ybuf;       // [T*S][d]   per-assignment down outputs before the combine
     uint32_t* rb_ctr;  // [ceil(d/rb4)] down item arrivals per row block (self-resetting)
     int32_t* hcs;      // [T*S]      sum of the hq codes of each assignment (tensor-core down)
-    int4* hmeta;       // [T*S]      reserved (no path writes it)
     uint8_t* xb;       // tensor-core operand B of gate/up: per task, activation rows in MMA layout
     uint8_t* hb;       // tensor-core operand B of down: per task, hq rows in MMA layout
     size_t bytes;
@@ -88,10 +87,10 @@ __host__ __device__ constexpr int tc_kc(int wb) { return 512 / wb; }
 __host__ __device__ constexpr int tc_kpad(int k, int wb) { return (k + tc_kc(wb) - 1) / tc_kc(wb) * tc_kc(wb); }
 // Bound on the padded rows of all tasks of a call: every task has >= 1 token
 // and pads by < 16 rows; tasks <= experts present + assignments / kTcNT.
-inline size_t tc_rows_bound(const Dims& m) {
+__host__ __device__ inline size_t tc_rows_bound(const Dims& m) {
     const size_t A = (size_t)m.T * m.S;
-    const size_t tasks = std::min(A, (size_t)(m.E + m.has_shared) + (A + kTcNT - 1) / kTcNT);
-    return A + 15 * tasks;
+    const size_t t2 = (size_t)(m.E + m.has_shared) + (A + kTcNT - 1) / kTcNT;
+    return A + 15 * (A < t2 ? A : t2);
 }
 // Rows per warp per work item of the gate/up and down kernels (one definition
 // for the kernels' template arguments and the host's item counts).
@@ -128,7 +127,6 @@ inline Ws ws_carve(const Dims& m, void* base) {
     w.ybuf = (float*)take(A * m.d * 4);
     w.rb_ctr = (uint32_t*)take((size_t)((m.d + kMinRowBlock4 - 1) / kMinRowBlock4) * 4);
     w.hcs = (int32_t*)take(A * 4);
-    w.hmeta = (int4*)take(A * 16);
     w.xb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.d, m.wb));
     w.hb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.f, m.wb));
     w.bytes = off;
@@ -166,6 +164,8 @@ struct Params {
     Ws ws;
     int a_cap;       // assignments the workspace layout holds (capacity T x S)
     unsigned long long* trace;  // optional per-CTA phase stamps of the decode kernel
+    unsigned long long wait_ns; // bound of the decode kernel's device-side waits (its slot waits: twice this)
+    int skip_h_task;            // testing: the one-token decode leaves this task's h unwritten (-1 = none)
     const float* w_router;
     const float* bias;
     float* out;
@@ -217,6 +217,22 @@ __device__ __forceinline__ void set_status(WsHeader* h, int code, int info) {
     if (atomicCAS(&h->status, 0, code) == 0) atomicExch(&h->status_info, info);
 }
 
+// Indices the kernels read from data -- routed experts, task lists,
+// assignment ids, padded-row offsets -- pass through idx_in(): it keeps v in
+// [lo, hi) so that no access leaves its buffer, whatever the data.  The
+// bounds-checked build of the library (compiled with MOE_BOUNDS,
+// libmoe_bounds.so) also records a value outside the range as MOE_EDEVICE
+// with the site code in the status word, which the tests read.
+__device__ __forceinline__ int idx_in(WsHeader* h, int v, int lo, int hi, int site) {
+#ifdef MOE_BOUNDS
+    if (v < lo || v >= hi) set_status(h, MOE_EDEVICE, site);
+#else
+    (void)h;
+    (void)site;
+#endif
+    return min(max(v, lo), hi - 1);
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier / bulk-copy / ordering wrappers (sm_90+ PTX, used on sm_100a)
 // ---------------------------------------------------------------------------
@@ -234,17 +250,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_u32(bar)) : "memory");
-}
-// Non-blocking test of a phase (try_wait may suspend the thread for a while
-// before it reports "not yet", which delays whatever else a polling loop does).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
@@ -276,20 +281,17 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 __device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_f32(float* p, float v) {
+    asm volatile("st.relaxed.gpu.global.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 // Morally strong (relaxed, gpu-scope) accesses for values that other CTAs poll
 // without a fence: each reader checks every value it uses against the preset
 // "not written" pattern, so no ordering between values is needed.
-constexpr uint32_t kNotWritten = 0x7fbadbadu;  // a NaN payload that arithmetic never produces
+constexpr uint32_t kNotWritten = 0x7fbadbadu;       // a NaN payload that arithmetic never produces
 constexpr uint32_t kCodesNotWritten = 0x80808080u;  // -128 bytes: never a code
-__device__ __forceinline__ void st_relaxed_f32(float* p, float v) {
-    asm volatile("st.relaxed.gpu.global.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
 __device__ __forceinline__ float ld_relaxed_f32(const float* p) {
     float v;
     asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
@@ -327,9 +329,6 @@ __device__ __forceinline__ void red_add_u32(uint32_t* p, uint32_t v) {
 }
 // Orders this thread's earlier global writes before its later ones at GPU scope.
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-// Orders generic-proxy accesses against async-proxy (bulk copy) accesses of the
-// same memory, e.g. codes stored by one CTA and bulk-copied by another.
-__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 __device__ __forceinline__ int ld_volatile_status(const WsHeader* h) {
     return *reinterpret_cast<const volatile int*>(&h->status);
 }
@@ -442,11 +441,12 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // Unlike the flag waits this does not stop early when another wait has already
 // failed: the slots' bulk copies must still be waited for, so that no copy is
 // in flight into shared memory when the CTA exits.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, WsHeader* hdr, int site,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             set_status(hdr, MOE_ETIMEOUT, site);
             return false;
         }
@@ -454,12 +454,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     return true;
 }
 // Wait until *flag == want (acquire), with the same bound.
-__device__ __forceinline__ bool flag_wait_bounded(const uint32_t* flag, uint32_t want, WsHeader* hdr, int site) {
+__device__ __forceinline__ bool flag_wait_bounded(const uint32_t* flag, uint32_t want, WsHeader* hdr, int site,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     if (ld_acquire_u32(flag) == want) return true;
     const uint64_t t0 = global_timer_ns();
     while (ld_acquire_u32(flag) != want) {
         if (ld_volatile_status(hdr) != 0) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             set_status(hdr, MOE_ETIMEOUT, site);
             return false;
         }

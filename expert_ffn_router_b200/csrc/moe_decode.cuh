@@ -238,7 +238,7 @@ __device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float
 // in registers; each round takes the largest selection score (lowest index on
 // ties) with two warp reductions.  Same rule and arithmetic as topk_warp.
 __device__ __forceinline__ void topk_warp_small(const uint2* prow, int E, int k, float scale, int& my_e,
-                                                float& my_w) {
+                                                float& my_w, unsigned long long* tr) {
     const int lane = threadIdx.x & 31;
     float sv[8];
     unsigned key[8];
@@ -250,6 +250,7 @@ __device__ __forceinline__ void topk_warp_small(const uint2* prow, int E, int k,
         sv[i] = __uint_as_float(pr[i].y);
         key[i] = lane + 32 * i < E ? float_key(__uint_as_float(pr[i].x)) : 0u;  // 0: below every real key
     }
+    if (tr && lane == 0 && key[0] != 1u) *tr = global_timer_ns();  // once loaded (the branch reads a value)
     float ssum = 0.0f, my_s = 0.0f;
     my_e = 0;
     for (int j = 0; j < k; ++j) {
@@ -350,7 +351,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         auto take = [&](uint32_t bytes) -> uint8_t* {
             if (pr > 0) {
                 const unsigned long long t0 = trace ? global_timer_ns() : 0;
-                mbar_wait_bounded(&C.empty[ps], (pr - 1) & 1, hdr, 100 + ps);
+                mbar_wait_bounded(&C.empty[ps], (pr - 1) & 1, hdr, 100 + ps, 2 * p.wait_ns);
                 if (trace) t_empty += global_timer_ns() - t0;
             }
             mbar_arrive_expect_tx(&C.full[ps], bytes);
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         };
         const int n_blobs = E + HS;
         auto issue_gu = [&](int blob, int j) {
-            blob = min(max(blob, 0), n_blobs - 1);  // never copy outside the pool, whatever happened
+            blob = idx_in(hdr, blob, 0, n_blobs, 611);  // never copy outside the pool, whatever happened
             const int r0 = j * kDecWarps, rows = min(kDecWarps, f - r0);  // f % 8 == 0: rows == 8
             const uint32_t bytes = (uint32_t)rows * rb_gu;
             const uint8_t* base = p.pool + (size_t)blob * p.blob_bytes;
@@ -398,7 +399,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             int ti = 0, j = c, jstep = G, jwrap = 0x7fffffff, sh_blob = E;
             if (ph == 1) {
                 DEC_TRACE(12);
-                mbar_wait_bounded(&C.route_ready, 0, hdr, 110);
+                mbar_wait_bounded(&C.route_ready, 0, hdr, 110, 2 * p.wait_ns);
                 DEC_TRACE(13);
                 n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
                 const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             // memory themselves, once written)
             const int n_rr = min(n_tasks, kDecRRMaxTasks);
             for (int ti = 0; ti < n_rr; ++ti) {
-                const int blob = min(max(C.tasks[ti].x, 0), n_blobs - 1);
+                const int blob = idx_in(hdr, C.tasks[ti].x, 0, n_blobs, 612);
                 const uint32_t wb = (uint32_t)rr_rows * rb_dn;
                 uint8_t* dst = take(wb + (uint32_t)rr_rows * 4);
                 bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)rr_lo * rb_dn, wb,
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             const long long lo = c * Nd / G, hi = (c + 1) * Nd / G;
             int ti = (int)(lo / pl.nu_dn), j = (int)(lo % pl.nu_dn);
             for (long long g = lo; g < hi; ++g) {
-                const int blob = min(max(C.tasks[ti].x, 0), n_blobs - 1);
+                const int blob = idx_in(hdr, C.tasks[ti].x, 0, n_blobs, 612);
                 const int r0 = j * pl.rd, rows = min(pl.rd, d - r0);  // multiples of 8
                 const uint32_t bytes = (uint32_t)rows * rb_dn;
                 uint64_t* bar = &C.full[ps];
@@ -460,7 +461,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         // the CTA and its shared memory) can retire
         for (int s = 0; s < nslot; ++s)
             if (issued > (uint32_t)s)
-                mbar_wait_bounded(&C.full[s], ((issued - s + nslot - 1) / nslot - 1) & 1, hdr, 120 + s);
+                mbar_wait_bounded(&C.full[s], ((issued - s + nslot - 1) / nslot - 1) & 1, hdr, 120 + s, 2 * p.wait_ns);
         DEC_TRACE(15);
         return;
     }
@@ -501,11 +502,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     };
     auto wait_full = [&]() -> const uint8_t* {
         const unsigned long long t0 = (trace && ctid == 0) ? global_timer_ns() : 0;
-        mbar_wait_bounded(&C.full[cs_slot], cs_phase, hdr, 200 + cs_slot);
+        mbar_wait_bounded(&C.full[cs_slot], cs_phase, hdr, 200 + cs_slot, 2 * p.wait_ns);
         if (trace && ctid == 0) t_full += global_timer_ns() - t0;
         return ring + (size_t)cs_slot * slot_bytes;
     };
-    auto release = [&]() {
+    auto release = [&]() {  // the proxy fence orders the warp's reads before the next bulk copy
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&C.empty[cs_slot]);
     };
@@ -702,7 +704,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
 #pragma unroll
             for (int i = 0; i < TM; ++i)
                 if (i < cur_n) {
-                    t_asg[i] = C.ttok[ti][i];
+                    t_asg[i] = idx_in(hdr, C.ttok[ti][i], 0, T * S, 613);
                     const int tok = t_asg[i] / S;
                     xoff[i] = tok * NSUB * nch_gu;
                     t_cs[i] = C.xcs[tok];
@@ -778,7 +780,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                         const float g = __fmul_rn((float)Gv, __fmul_rn(sg, t_sx[i]));
                         const float uu = __fmul_rn((float)Uv, __fmul_rn(su, t_sx[i]));
                         const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), uu);
-                        st_relaxed_f32(p.ws.h + (size_t)t_asg[i] * f + r, h);
+                        // (the h-skip test hook exists only on the row-range path)
+                        if (TM > 1 || ND == 0 || cur_task != p.skip_h_task)
+                            st_relaxed_f32(p.ws.h + (size_t)t_asg[i] * f + r, h);
                         amax[i] = fmaxf(amax[i], fabsf(h));
                     }
                 }
@@ -803,7 +807,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         int ti = 0, j = c, jstep = G, jwrap = 0x7fffffff;  // shared: units c, c + G, ... of task 0
         if (ph == 1) {
             // ---- 4. grid barrier, then every CTA derives the routing ----
-            if (ctid == 0) flag_wait_bounded(&hdr->b1_gen, epoch + 1, hdr, 300);
+            if (ctid == 0) flag_wait_bounded(&hdr->b1_gen, epoch + 1, hdr, 300, p.wait_ns);
             named_sync(kDecBar, kDecCons);
             if (ctid == 0) DEC_TRACE(4);
             if (c == 0 && ctid == 0) hdr->epoch = epoch + 1;
@@ -812,13 +816,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 float my_w;
                 if (E <= kDecBiasCache) {
                     topk_warp_small(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale,
-                                    my_e, my_w);
+                                    my_e, my_w, trace && warp == 0 ? trace + 18 : nullptr);
                 } else {
                     float* scr = reinterpret_cast<float*>(hsb) + (size_t)warp * 2 * E;
                     topk_warp(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale, scr,
                               scr + E, my_e, my_w);
                 }
                 if (lane < k) {
+                    my_e = idx_in(hdr, my_e, 0, E, 618);
                     C.idx[warp][lane] = my_e;
                     C.w[warp][lane] = my_w;
                     if (c == 0) {
@@ -909,7 +914,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             // max |h| over the row, then the codes and the scale, with relaxed
             // stores that the down units poll in turn (no count, no fence)
             for (int ti = c; ti < n_tasks; ti += G) {
-                const int a = min(max(C.ttok[ti][0], 0), S - 1);
+                const int a = idx_in(hdr, C.ttok[ti][0], 0, S, 615);
                 const int pc = ctid;
                 float4 hv4[4];
                 float m = 0.0f;
@@ -925,7 +930,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                                  __float_as_uint(hv4[q4].z) != kNotWritten && __float_as_uint(hv4[q4].w) != kNotWritten;
                         }
                         if (ok) break;
-                        if (global_timer_ns() - t0 > kWaitLimitNs || ld_volatile_status(hdr) != 0) {
+                        if (global_timer_ns() - t0 > p.wait_ns || ld_volatile_status(hdr) != 0) {
                             set_status(hdr, MOE_ETIMEOUT, 410);
                             break;
                         }
@@ -966,7 +971,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             for (int ti = 0; ti < min(n_tasks, kDecRRMaxTasks); ++ti, next_unit()) {
                 if (!mine()) continue;
                 const uint8_t* slot = wait_full();
-                const int a = min(max(C.ttok[ti][0], 0), S - 1);
+                const int a = idx_in(hdr, C.ttok[ti][0], 0, S, 615);
                 // the task's scale and codes straight from global memory, each
                 // polled until written (the whole code row sits in the warp)
                 float shv = 0.0f;
@@ -986,8 +991,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                                        has_byte_80(hrr[i][sb].w);
                             }
                         if (!__any_sync(kFull, bad != 0u)) break;
-                        if (global_timer_ns() - t0 > kWaitLimitNs || ld_volatile_status(hdr) != 0) {
-                            set_status(hdr, MOE_ETIMEOUT, 420);
+                        // give up as a warp (lanes may read the clock or the status differently)
+                        const bool give_up = global_timer_ns() - t0 > p.wait_ns || ld_volatile_status(hdr) != 0;
+                        if (__any_sync(kFull, give_up)) {
+                            if (lane == 0) set_status(hdr, MOE_ETIMEOUT, 420);
                             break;
                         }
                     }
@@ -1061,10 +1068,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         const int n = C.tasks[ti].y;
         if (ti != C.hq_task[grp]) {  // requantise and stage this task's h (the whole group agrees on ti)
             named_sync(2 + grp, kDecGrp);
-            if (gtid == 0) flag_wait_bounded(rows_cur + ti, (uint32_t)(pl.nu_gu * kDecWarps), hdr, 400);
+            if (gtid == 0) flag_wait_bounded(rows_cur + ti, (uint32_t)(pl.nu_gu * kDecWarps), hdr, 400, p.wait_ns);
             named_sync(2 + grp, kDecGrp);
             for (int i = 0; i < n; ++i) {
-                const int a = C.ttok[ti][i];
+                const int a = idx_in(hdr, C.ttok[ti][i], 0, T * S, 614);
                 const float m = __uint_as_float(__ldcg(amax_cur + a));
                 const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
                 const float rh = quant_recip(sh);
@@ -1131,7 +1138,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 for (int i = 0; i < ND; ++i) dot_chunk_regs<WB>(wv[q][i], hr[i], a0, a1);
                 dv[q] = a0 + a1;
             }
-            const int a = C.ttok[ti][0];
+            const int a = idx_in(hdr, C.ttok[ti][0], 0, T * S, 616);
 #pragma unroll
             for (int q = 0; q < kDecNQ; ++q) {
                 const int D = __reduce_add_sync(kFull, dv[q]) - code_offset<WB>() * C.hcs[grp][0];
@@ -1170,7 +1177,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 if (i < n) {
                     const int D = __reduce_add_sync(kFull, acc[i]) - code_offset<WB>() * C.hcs[grp][i];
                     if (lane == i) {
-                        const int a = C.ttok[ti][i];
+                        const int a = idx_in(hdr, C.ttok[ti][i], 0, T * S, 617);
                         p.ws.ybuf[(size_t)a * d + r] = __fmul_rn((float)D, __fmul_rn(sdr, C.hsh[grp][i]));
                     }
                 }

@@ -36,12 +36,12 @@ __global__ void __launch_bounds__(kThreads) k_gate_up(const Params p) {
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int ti = item / p.nrb3, rb = item % p.nrb3;
         const int4 task = p.ws.tasks[ti];
-        const int n = task.z;
+        const int n = idx_in(p.ws.hdr, task.z, 0, CH + 1, 621);
         __syncthreads();  // previous item done with the staged rows
         if (warp == 0) {
             int a = -1, tok = -1;
             if (lane < n) {
-                a = p.ws.asg[task.y + lane];
+                a = idx_in(p.ws.hdr, p.ws.asg[idx_in(p.ws.hdr, task.y + lane, 0, p.a_cap, 622)], 0, p.a_cap, 623);
                 tok = a / S;
             }
             const bool same = __all_sync(kFull, s_n == n && (lane >= n || s_tok[lane] == tok));
@@ -67,8 +67,9 @@ __global__ void __launch_bounds__(kThreads) k_gate_up(const Params p) {
             __syncthreads();
             if (tid == 0) s_n = nn;
         }
-        const uint8_t* blob = p.pool + (size_t)task.x * p.blob_bytes;
-        const float* sc = p.scales + (size_t)task.x * p.scale_rows;
+        const int bx = idx_in(p.ws.hdr, task.x, 0, p.m.E + p.m.has_shared, 624);
+        const uint8_t* blob = p.pool + (size_t)bx * p.blob_bytes;
+        const float* sc = p.scales + (size_t)bx * p.scale_rows;
         float amax[CH];
 #pragma unroll
         for (int t = 0; t < CH; ++t) amax[t] = 0.0f;
@@ -192,10 +193,11 @@ __global__ void __launch_bounds__(kThreads) k_down(const Params p) {
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         const int ti = item / p.nrb4, rb = item % p.nrb4;
         const int4 task = p.ws.tasks[ti];
-        const int n = task.z;
+        const int n = idx_in(p.ws.hdr, task.z, 0, CH + 1, 631);
         __syncthreads();
         if (s_key != ti) {  // stage this task's h codes
-            if (tid < n) s_asg[tid] = p.ws.asg[task.y + tid];
+            if (tid < n)
+                s_asg[tid] = idx_in(p.ws.hdr, p.ws.asg[idx_in(p.ws.hdr, task.y + tid, 0, p.a_cap, 632)], 0, p.a_cap, 633);
             __syncthreads();
             for (int i = 0; i < n; ++i) {
                 const int a = s_asg[i];
@@ -210,8 +212,9 @@ __global__ void __launch_bounds__(kThreads) k_down(const Params p) {
             if (tid == 0) s_key = ti;
             __syncthreads();
         }
-        const uint8_t* wd = p.pool + (size_t)task.x * p.blob_bytes + 2 * (size_t)f * (d * WB / 8);
-        const float* sd = p.scales + (size_t)task.x * p.scale_rows + 2 * f;
+        const int bx = idx_in(p.ws.hdr, task.x, 0, p.m.E + p.m.has_shared, 634);
+        const uint8_t* wd = p.pool + (size_t)bx * p.blob_bytes + 2 * (size_t)f * (d * WB / 8);
+        const float* sd = p.scales + (size_t)bx * p.scale_rows + 2 * f;
         const int r0 = rb * RB + warp * RPW;
         uint4 wv[RPW][NCL];
 #pragma unroll

@@ -193,17 +193,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
                 const int ti = u / nrb, rb = u - ti * nrb;
                 const int4 task = p.ws.tasks[ti];
-                const int npad = tc_npad(task.z);
+                const int npad = tc_npad(idx_in(hdr, task.z, 1, kTcNT + 1, 641));
                 const uint32_t bbytes = (uint32_t)npad * KC;
+                const int bx = idx_in(hdr, task.x, 0, p.m.E + p.m.has_shared, 642);
                 int y0, y1;
                 if (EPI == 0) {
-                    y0 = task.x * 3 * f + rb * 128;
+                    y0 = bx * 3 * f + rb * 128;
                     y1 = y0 + f;
                 } else {
-                    y0 = task.x * 3 * d + 2 * d + rb * 256;
+                    y0 = bx * 3 * d + 2 * d + rb * 256;
                     y1 = y0 + 128;
                 }
-                const uint8_t* bsrc = bbuf + (size_t)task.w * kpad;
+                const uint8_t* bsrc =
+                    bbuf + (size_t)idx_in(hdr, task.w, 0, (int)tc_rows_bound(p.m) - npad + 1, 643) * kpad;
                 for (int c = 0; c < nch; ++c) {
                     if (!tc_wait(&ctl->empty[slot], ph ^ 1u, hdr, 0x7101)) {
                         ok = false;
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool ok = true, issued = false;
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++uidx) {
                 const int ti = u / nrb;
-                const int npad = tc_npad(p.ws.tasks[ti].z);
+                const int npad = tc_npad(idx_in(hdr, p.ws.tasks[ti].z, 1, kTcNT + 1, 644));
                 const uint32_t idesc = tc_idesc_u8s8(npad);
                 const uint32_t lbo = (uint32_t)npad * 16;
                 const uint32_t buf = uidx & 1u;
@@ -302,6 +304,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc_unpack_tile<WB>(sp + kTcBox, row, hh, acol + ACOLS);
                     tmem_st_wait();
                 }
+                // this warp's reads of the slot (generic proxy) before the
+                // producer's next TMA load into it (async proxy), which the
+                // MMA's commit of this chunk lets it issue
+                fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->afull[ab]);
@@ -326,11 +332,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++uidx) {
             const int ti = u / nrb, rb = u - ti * nrb;
             const int4 task = p.ws.tasks[ti];
-            const int n = task.z, npad = tc_npad(n);
+            const int n = idx_in(hdr, task.z, 1, kTcNT + 1, 645), npad = tc_npad(n);
+            const int bx = idx_in(hdr, task.x, 0, p.m.E + p.m.has_shared, 648);
             const uint32_t buf = uidx & 1u;
             named_sync(2, kTcEpi);  // the previous unit's metadata is no longer read
             if (etid < n) {
-                const int a = p.ws.asg[task.y + etid];
+                const int a = idx_in(hdr, p.ws.asg[idx_in(hdr, task.y + etid, 0, p.a_cap, 646)], 0, p.a_cap, 647);
                 ctl->asg[etid] = a;
                 if (EPI == 0) {
                     const int tok = a / p.m.S;
@@ -349,8 +356,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (ok && EPI == 0) {
                 const int r = rb * 128 + row;
                 const bool rv = r < f;
-                const float sg = rv ? __ldg(p.scales + (size_t)task.x * p.scale_rows + r) : 0.0f;
-                const float su = rv ? __ldg(p.scales + (size_t)task.x * p.scale_rows + f + r) : 0.0f;
+                const float sg = rv ? __ldg(p.scales + (size_t)bx * p.scale_rows + r) : 0.0f;
+                const float su = rv ? __ldg(p.scales + (size_t)bx * p.scale_rows + f + r) : 0.0f;
                 for (int tg = 0; tg * 8 < npad; ++tg) {
                     int G[8], U[8];
                     tmem_ld8(dcol + tg * 8, G);
@@ -380,7 +387,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             } else if (ok) {
                 const int r0 = rb * 256 + row;
-                const float* sd = p.scales + (size_t)task.x * p.scale_rows + 2 * f;
+                const float* sd = p.scales + (size_t)bx * p.scale_rows + 2 * f;
                 const float s0 = r0 < d ? __ldg(sd + r0) : 0.0f;
                 const float s1 = r0 + 128 < d ? __ldg(sd + r0 + 128) : 0.0f;
                 float* dst = p.direct_out ? p.out : p.ws.ybuf;
@@ -440,9 +447,11 @@ __global__ void __launch_bounds__(kThreads) k_tc_requant(const Params p) {
             else hi = mid - 1;
         }
         const int4 task = __ldg(p.ws.tasks + lo);
-        const int j = R - task.w, npad = tc_npad(task.z);
+        const int j = idx_in(p.ws.hdr, R - task.w, 0, kTcNT + 16, 651), npad = tc_npad(task.z);
         const bool live = j < task.z;
-        const int a = live ? __ldg(p.ws.asg + task.y + j) : 0;
+        const int a = live ? idx_in(p.ws.hdr, __ldg(p.ws.asg + idx_in(p.ws.hdr, task.y + j, 0, p.a_cap, 652)), 0,
+                                    p.a_cap, 653)
+                           : 0;
         const float m = live ? __uint_as_float(__ldcg(p.ws.amax + a)) : 0.0f;
         const float sh = m == 0.0f ? 0.0f : __fdiv_rn(m, 127.0f);
         const float rh = quant_recip(sh);
@@ -498,8 +507,10 @@ __global__ void __launch_bounds__(kThreads) k_tc_gather(const Params p, const in
             else hi = mid - 1;
         }
         const int4 task = __ldg(p.ws.tasks + lo);
-        const int j = R - task.w, npad = tc_npad(task.z);
-        const int key = j < task.z ? __ldg(p.ws.asg + task.y + j) / key_div : -1;
+        const int j = idx_in(p.ws.hdr, R - task.w, 0, kTcNT + 16, 654), npad = tc_npad(task.z);
+        const int key = j < task.z ? idx_in(p.ws.hdr, __ldg(p.ws.asg + idx_in(p.ws.hdr, task.y + j, 0, p.a_cap, 655)),
+                                            0, p.a_cap, 656) / key_div
+                                   : -1;
         const int8_t* row = src + (size_t)(key < 0 ? 0 : key) * ld;
         uint8_t* out = dst + (size_t)task.w * kpad;
 #pragma unroll 4

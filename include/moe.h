@@ -128,9 +128,11 @@ MOE_API moe_status moe_route(const moe_config* cfg, const void* x, moe_dtype dty
  * keeps until the process exits; the call allocates nothing.
  *  - Limits: T <= 8 tokens, n_experts <= 1024, top_k <= 32; larger requests
  *    return MOE_EINVAL with a message naming the limit.
- *  - The first call on each device looks up that array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *  - Each call looks up that array's device address on the current device
+ *    (cudaGetSymbolAddress, with that device current; nothing is kept between
+ *    calls, so a device reset by the caller is harmless).  The first call on
+ *    a device also loads the library's device code there: make that first
+ *    call before any stream capture.
  *  - Every call, on every stream, shares the one array: calls whose work
  *    overlaps on the GPU race and give undefined results.  Each call clears
  *    the control word it needs at its start. */
@@ -186,11 +188,12 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *         (ns) at its phase boundaries: [0] start, [1] tokens quantised,
  *         [2] router rows done, [3] shared-expert gate/up done, [4] grid
  *         barrier passed, [5] routing derived, [6] routed gate/up done,
- *         [7] first down staging ready, [8] down done, [11] top-k done;
+ *         [7] first down staging ready, [8] down done, [11] top-k done,
+ *         [18] router logits loaded for the top-k (first warp);
  *         totals: [9] consumer wait for data, [10] producer wait for slots;
  *         producer: [12] rows known before routing issued, [13] routing
- *         received, [14] all rows issued, [15] all copies landed; single-token
- *         down: [16] the CTA's designated task's h row complete (polled),
+ *         received, [14] all rows issued, [15] all copies landed; one-token
+ *         row-range down: [16] the CTA's designated task's h row complete (polled),
  *         [17] its codes and scale written, [20] first down unit's codes
  *         seen, [21] last down unit done.  Untouched entries are left as
  *         is. */
@@ -201,7 +204,18 @@ typedef struct {
     int32_t n_launches;
     void* trace;
     int32_t path_ran;
-    int32_t reserved[3];
+    /* in: bound of the decode kernel's device-side waits in microseconds
+     * (0 = 2 s; its waits for ring slots take twice this, so that a stalled
+     * hand-off reports before the slot waits behind it); a wait that runs out
+     * records MOE_ETIMEOUT with a site code (moe_poll_status) and the kernel
+     * finishes without the missing data. */
+    int32_t wait_limit_us;
+    /* in, for tests of the bounded waits: 1 + t makes the one-token decode
+     * with row-range down (the GLM-5.2 expert shapes) leave task t's h values
+     * unwritten (task 0 is the shared expert when there is one, then the
+     * routed experts in ascending id order), so that every wait on them runs
+     * out; ignored on every other path; 0 = off. */
+    int32_t test_skip_h;
 } moe_layer_opts;
 
 /* moe_layer with options (opts may be NULL, then identical to moe_layer). */

@@ -86,3 +86,26 @@ def test_expert_entry_points_validate():
 def test_status_strings():
     for st in (0, -1, -2, -3, -4, -5, -6):
         assert L.moe_status_string(st).decode().startswith("MOE_")
+
+
+def test_bounds_checked_build_exports_the_same_symbols():
+    import os
+    path = os.path.join(os.path.dirname(M.LIB_PATH), "libmoe_bounds.so")
+    assert os.path.exists(path), "libmoe_bounds.so is not built"
+    B = ctypes.CDLL(path)
+    for n in M.declared_symbols():
+        assert hasattr(B, n), n
+
+
+def test_layer_opts_rejects_negative_test_fields():
+    c = good_cfg()
+    pool = M.MoePool(FAKE, FAKE)
+    o = M.MoeLayerOpts()
+    o.wait_limit_us = -1
+    st = L.moe_layer_ex(ctypes.byref(c), ctypes.byref(pool), FAKE, FAKE, FAKE, 0, 4, FAKE, 0, None, None, FAKE,
+                        1 << 40, None, ctypes.byref(o))
+    assert st == M.MOE_EINVAL
+    o.wait_limit_us, o.test_skip_h = 0, -3
+    st = L.moe_layer_ex(ctypes.byref(c), ctypes.byref(pool), FAKE, FAKE, FAKE, 0, 4, FAKE, 0, None, None, FAKE,
+                        1 << 40, None, ctypes.byref(o))
+    assert st == M.MOE_EINVAL
