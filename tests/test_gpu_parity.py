@@ -33,6 +33,19 @@ SMALL = {
 }
 PATHS = {"auto": M.MOE_PATH_AUTO, "multi": M.MOE_PATH_MULTI}
 
+# One-token decode on small pools of d = 2048 (the decode kernel's runtime-loop
+# rows): int4 and int2 rows, no shared expert, E > 256 (its shared-memory
+# top-k) and k = 32.
+SINGLE = {
+    "s1_int4": W.workload(0).replace(name="s1_int4", d=2048, f=1024, n_experts=16, top_k=4, T=1, x_dtype="bf16"),
+    "s1_int2": W.workload(0).replace(name="s1_int2", d=2048, f=2048, n_experts=24, top_k=5, T=1, wbits=2,
+                                     x_dtype="bf16"),
+    "s1_no_shared": W.workload(0).replace(name="s1_no_shared", d=2048, f=1024, n_experts=12, top_k=3, T=1,
+                                          has_shared=0),
+    "s1_E512": W.workload(0).replace(name="s1_E512", d=2048, f=1024, n_experts=512, top_k=8, T=1),
+    "s1_k32": W.workload(0).replace(name="s1_k32", d=2048, f=1024, n_experts=64, top_k=32, T=1),
+}
+
 
 def cfg_of(wl):
     return M.config(wl.d, wl.f, wl.n_experts, wl.top_k, wl.has_shared, wl.wbits, wl.routed_scale)
@@ -223,29 +236,37 @@ def test_layer_decode_repeats_bit_identical():
     for bit.  Its gate/up -> down hand-off has no fence (readers poll values
     preset to "not written"), so a stale or torn read would show here as a
     differing output (the outputs' agreement with the oracle is
-    test_layer_decode_full_size's)."""
+    test_layer_decode_full_size's; each token's first output, the reference
+    of the repeats, is also checked against the oracle here, so that a race
+    on a first call cannot set a wrong reference)."""
     wl = W.workload(1)
-    dl = W.device_layer(wl, 0, 0)
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
     cfg = cfg_of(wl)
     pool = M.make_pool(dl.pool_w, dl.pool_s)
     ws = M.workspace(cfg, 1)
     out = torch.empty(1, wl.d, device="cuda")
+    idx = torch.empty(1, wl.top_k, dtype=torch.int32, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    toks = [to_dev(x_host(wl, s)) for s in range(6)]
-    refs, bad = {}, 0
+    xs = [x_host(wl, s) for s in range(6)]
+    toks = [to_dev(x) for x in xs]
+    refs, ref_idx, bad = {}, {}, 0
     for it in range(300):
         i = it % 6
         if it % 2 == 0:
             flush.fill_(it & 0xFF)
-        M.moe_layer(cfg, pool, dl.w_router, dl.bias, toks[i], out, ws)
+        M.moe_layer(cfg, pool, dl.w_router, dl.bias, toks[i], out, ws, topk_idx_out=idx)
         o = out.clone()
         if i in refs:
             bad += int(not torch.equal(o, refs[i]))
         else:
             refs[i] = o
+            ref_idx[i] = idx.cpu().numpy().copy()
     torch.cuda.synchronize()
     assert_ok(ws)
     assert bad == 0
+    for i in range(6):
+        compare_layer(wl, L, xs[i], refs[i], ref_idx[i])
 
 
 def test_layer_decode_int2_full_size():
@@ -328,3 +349,30 @@ def test_workspace_reuse_and_status():
     torch.cuda.synchronize()
     assert torch.equal(outs[0], ref) and torch.equal(outs[3], ref)  # deterministic
     assert torch.equal(outs[2], outs[4])
+
+
+@pytest.mark.parametrize("name", list(SINGLE))
+def test_layer_one_token_small_pools(name):
+    """One token through the decode kernel on small pools (its runtime-loop
+    rows; E up to 512, top-k up to 32): 6 tokens in turn on one workspace,
+    each against the oracle; then the accumulate mode."""
+    wl = SINGLE[name]
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    cfg = cfg_of(wl)
+    pool = M.make_pool(dl.pool_w, dl.pool_s)
+    ws = M.workspace(cfg, 1)
+    for s_ in range(6):
+        x = x_host(wl, s_)
+        out = torch.empty(1, wl.d, device="cuda")
+        idx = torch.empty(1, wl.top_k, dtype=torch.int32, device="cuda")
+        o = M.MoeLayerOpts()
+        M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x), out, ws, topk_idx_out=idx, opts=o)
+        assert_ok(ws)
+        assert o.path_ran == M.MOE_PATH_DECODE
+        compare_layer(wl, L, x, out, idx.cpu().numpy())
+    base = torch.randn(1, wl.d, device="cuda")
+    acc = base.clone()
+    M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x), acc, ws, accumulate=True)
+    assert_ok(ws)
+    np.testing.assert_allclose(acc.cpu().numpy(), (base + out).cpu().numpy(), rtol=1e-6, atol=1e-5)
