@@ -22,7 +22,7 @@ import workloads as W  # noqa: E402
 
 
 def args_for(workload, steps=2, warmup=3, gpus=1):
-    return argparse.Namespace(steps=steps, warmup=warmup, gpus=gpus, workload=workload)
+    return argparse.Namespace(steps=steps, warmup=warmup, gpus=gpus, workload=workload, layers=0)
 
 
 def run_reference(workload, monkeypatch, rank="0"):
