@@ -302,11 +302,12 @@ def reference_arm(args, wl):
 # GPU arm
 # ---------------------------------------------------------------------------
 TRACE_NAMES = {0: "start", 1: "quantised", 2: "router_done", 3: "shared_gate_up_done", 4: "grid_barrier",
-               5: "routing_done", 6: "routed_gate_up_done", 7: "first_down_staged", 8: "down_done",
+               5: "routing_done", 6: "routed_gate_up_done", 7: "designated_requant_done", 8: "down_done",
                9: "cons_wait_full_total", 10: "prod_wait_empty_total", 11: "topk_done",
                12: "prod_pre_routing_issued", 13: "prod_routing_received", 14: "prod_all_issued",
                15: "prod_drained", 16: "designated_h_row_complete", 17: "designated_codes_written",
-               18: "topk_values_loaded", 20: "first_down_codes_seen", 21: "last_down_unit_done"}
+               18: "topk_values_loaded", 20: "all_codes_staged", 21: "last_down_unit_done",
+               22: "first_down_unit_done"}
 
 
 def write_trace(path, M, cfg, pool, dl, xbuf, out, ws, dev, flush_l2):

@@ -30,8 +30,10 @@
 //      requantises them into int8 codes in the dot layout (max |h| from the
 //      values themselves) and writes codes and scale; every CTA owns a
 //      contiguous range of output rows, streams those rows of every task's
-//      down matrix, polls the task's codes and scale straight from global
-//      memory, and combines its rows locally;
+//      down matrix (each CTA starting at its own task, so that the CTAs read
+//      different matrices at once), stages every task's codes and scale in
+//      shared memory in one batch of polled loads, and combines its rows
+//      locally;
 //   6. otherwise: down units (waiting, bounded, until their task's counter
 //      shows every gate/up row) requantise and stage the task's h; at the end
 //      each CTA signs its row blocks off and the CTA bringing a row block's
@@ -71,13 +73,18 @@ struct DecPlan {
     int xs_off, hs_off, ring_off, smem_bytes;
     int hs_grp_bytes;  // h staging bytes of one consumer group (T * f)
     int rowrange;      // single-token down by output-row ranges (see step 6r)
+    int dn_rot;        // row-range: CTA c takes the down tasks from task c mod n_tasks on
 };
 // Row-range down unit (single token): [rows x down row][row scales at wbytes].
 constexpr int kDecRRMaxRows = 44;
 
 constexpr int kDecRRMaxTasks = kDecMaxK + 1;  // tasks of a single token (row-range down)
+constexpr int kDecRRChunks = 3;  // row-range: 16-byte chunks of the tasks' codes each consumer thread stages
 
+// Shared control block of the kernel, sized for TM tokens.
+template <int TM>
 struct DecCtl {
+    static constexpr int kTasks = TM * kDecMaxK + 1;  // the shared expert + one task per (token, slot) at most
     uint64_t full[kDecMaxSlots];
     uint64_t empty[kDecMaxSlots];
     uint64_t route_ready;
@@ -85,21 +92,22 @@ struct DecCtl {
     int n_tasks;
     int hq_task[kDecGroups];
     int n_last;
-    float sx[kDecMaxT];
-    int xcs[kDecMaxT];
-    int idx[kDecMaxT][kDecMaxK];
-    float w[kDecMaxT][kDecMaxK];
-    int4 tasks[kDecMaxTasks];  // (blob, n tokens, -, -)
-    int ttok[kDecMaxTasks][kDecMaxT];
-    int sorted[kDecMaxT * kDecMaxK];    // assignment ids by (expert, token, slot)
-    int sorted_e[kDecMaxT * kDecMaxK];  // their experts
-    int hcs[kDecGroups][kDecMaxT];
-    float hsh[kDecGroups][kDecMaxT];
+    float sx[TM];
+    int xcs[TM];
+    int idx[TM][kDecMaxK];
+    float w[TM][kDecMaxK];
+    int4 tasks[kTasks];  // (blob, n tokens, -, -)
+    int ttok[kTasks][TM];
+    int sorted[TM * kDecMaxK];    // assignment ids by (expert, token, slot)
+    int sorted_e[TM * kDecMaxK];  // their experts
+    int hcs[kDecGroups][TM];
+    float hsh[kDecGroups][TM];
     int last_rb[kDecCons];
     float bias_s[kDecBiasCache];  // the router bias (E <= kDecBiasCache)
     float redf[kDecConsWarps];
     int redi[kDecConsWarps];
-    float part[kDecGroups][kDecWarps][2 * kDecMaxT];
+    float part[kDecGroups][kDecWarps][2 * TM];
+    float rsh[kDecRRMaxTasks];  // one token: the scale of each task's staged codes
 };
 
 // --- consumer reductions over all consumer warps (named barrier 1) ---------
@@ -288,7 +296,8 @@ template <int WB, int TM, int NG, int ND, typename XT>
 __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const DecPlan pl, const XT* __restrict__ x) {
     constexpr int NSUB = 8 / WB;
     extern __shared__ __align__(128) uint8_t dec_smem[];
-    DecCtl& C = *reinterpret_cast<DecCtl*>(dec_smem);
+    DecCtl<TM>& C = *reinterpret_cast<DecCtl<TM>*>(dec_smem);
+    constexpr int kTasks = DecCtl<TM>::kTasks;
     uint4* xs = reinterpret_cast<uint4*>(dec_smem + pl.xs_off);
     uint8_t* hsb = dec_smem + pl.hs_off;
     uint8_t* ring = dec_smem + pl.ring_off;
@@ -401,7 +410,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 DEC_TRACE(12);
                 mbar_wait_bounded(&C.route_ready, 0, hdr, 110, 2 * p.wait_ns);
                 DEC_TRACE(13);
-                n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
+                n_tasks = min(max(C.n_tasks, HS), kTasks);
                 const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
                 const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
                 n_units = hi - lo;
@@ -425,7 +434,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             // their scales (the consumers read the task's codes from global
             // memory themselves, once written)
             const int n_rr = min(n_tasks, kDecRRMaxTasks);
-            for (int ti = 0; ti < n_rr; ++ti) {
+            const int rot = pl.dn_rot ? c % n_rr : 0;  // the CTA's task order (so the CTAs read different matrices)
+            for (int i = 0; i < n_rr; ++i) {
+                const int ti = i + rot < n_rr ? i + rot : i + rot - n_rr;
                 const int blob = idx_in(hdr, C.tasks[ti].x, 0, n_blobs, 612);
                 const uint32_t wb = (uint32_t)rr_rows * rb_dn;
                 uint8_t* dst = take(wb + (uint32_t)rr_rows * 4);
@@ -880,7 +891,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 mbar_arrive(&C.route_ready);  // the producer may issue routed rows
                 DEC_TRACE(5);
             }
-            n_tasks = min(max(C.n_tasks, HS), kDecMaxTasks);
+            n_tasks = min(max(C.n_tasks, HS), kTasks);
             n_units = n_sh_units - n_sh_first;
             j = c + n_sh_first * G;
         } else if (ph == 2) {
@@ -964,42 +975,67 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 }
             }
             if (ctid == 0) DEC_TRACE(7);
-            // down units: one per task, this CTA's rows; y of (assignment, row)
-            // kept in shared memory for the combine
-            float* ys = reinterpret_cast<float*>(hsb);  // [S][kDecNQ * kDecWarps]
+            // stage the codes of every task at once: each consumer thread
+            // polls up to kDecRRChunks 16-byte chunks (and one thread per
+            // task the scale) until written, into shared memory; then one
+            // down unit per task in the CTA's task order, with nothing but
+            // its weight rows to wait for.  y of (assignment, row) stays in
+            // shared memory for the combine.
             constexpr int RRW = kDecNQ * kDecWarps;
-            for (int ti = 0; ti < min(n_tasks, kDecRRMaxTasks); ++ti, next_unit()) {
-                if (!mine()) continue;
-                const uint8_t* slot = wait_full();
-                const int a = idx_in(hdr, C.ttok[ti][0], 0, S, 615);
-                // the task's scale and codes straight from global memory, each
-                // polled until written (the whole code row sits in the warp)
+            const int n_rr = min(n_tasks, kDecRRMaxTasks);
+            const int cpt = f / 16;      // code chunks per task
+            const int nq = n_rr * cpt;   // <= kDecRRChunks * kDecCons (the plan checks)
+            uint4* stage = reinterpret_cast<uint4*>(hsb);               // [n_rr][f] codes
+            float* ys = reinterpret_cast<float*>(hsb + (size_t)S * f);  // [S][RRW]
+            {
+                uint4 cv[kDecRRChunks];
                 float shv = 0.0f;
-                uint4 hrr[ND][NSUB];
-                {
-                    const uint4* hq4 = reinterpret_cast<const uint4*>(p.ws.hq + (size_t)a * f);
-                    const uint64_t t0 = global_timer_ns();
-                    for (;;) {
-                        shv = ld_relaxed_f32(p.ws.sh + a);
-                        uint32_t bad = __float_as_uint(shv) == kNotWritten;
+                const uint64_t t0 = global_timer_ns();
+                for (;;) {
+                    uint32_t bad = 0u;
 #pragma unroll
-                        for (int i = 0; i < ND; ++i)
-#pragma unroll
-                            for (int sb = 0; sb < NSUB; ++sb) {
-                                hrr[i][sb] = ld_relaxed_u4(hq4 + sb * nch_dn + lane + 32 * i);
-                                bad |= has_byte_80(hrr[i][sb].x) | has_byte_80(hrr[i][sb].y) | has_byte_80(hrr[i][sb].z) |
-                                       has_byte_80(hrr[i][sb].w);
-                            }
-                        if (!__any_sync(kFull, bad != 0u)) break;
-                        // give up as a warp (lanes may read the clock or the status differently)
-                        const bool give_up = global_timer_ns() - t0 > p.wait_ns || ld_volatile_status(hdr) != 0;
-                        if (__any_sync(kFull, give_up)) {
-                            if (lane == 0) set_status(hdr, MOE_ETIMEOUT, 420);
-                            break;
+                    for (int r = 0; r < kDecRRChunks; ++r) {
+                        const int q = ctid + r * kDecCons;
+                        if (q < nq) {
+                            const int a = idx_in(hdr, C.ttok[q / cpt][0], 0, S, 615);
+                            cv[r] = ld_relaxed_u4(reinterpret_cast<const uint4*>(p.ws.hq + (size_t)a * f) + q % cpt);
+                            bad |= has_byte_80(cv[r].x) | has_byte_80(cv[r].y) | has_byte_80(cv[r].z) | has_byte_80(cv[r].w);
                         }
                     }
+                    if (ctid < n_rr) {
+                        shv = ld_relaxed_f32(p.ws.sh + idx_in(hdr, C.ttok[ctid][0], 0, S, 615));
+                        bad |= __float_as_uint(shv) == kNotWritten;
+                    }
+                    if (bad == 0u) break;
+                    if (global_timer_ns() - t0 > p.wait_ns || ld_volatile_status(hdr) != 0) {
+                        set_status(hdr, MOE_ETIMEOUT, 420);
+                        break;
+                    }
+                    __nanosleep(64);
                 }
-                if (ti == 0 && gtid == 0) DEC_TRACE(20);
+#pragma unroll
+                for (int r = 0; r < kDecRRChunks; ++r) {
+                    const int q = ctid + r * kDecCons;
+                    if (q < nq) stage[q] = cv[r];
+                }
+                if (ctid < n_rr) C.rsh[ctid] = shv;
+            }
+            named_sync(kDecBar, kDecCons);  // every task's codes and scale are staged
+            if (ctid == 0) DEC_TRACE(20);
+            const int rot = pl.dn_rot ? c % n_rr : 0;
+            int n_done = 0;  // down units group 0 has finished (traced)
+            for (int i = 0; i < n_rr; ++i, next_unit()) {
+                if (!mine()) continue;
+                const int ti = i + rot < n_rr ? i + rot : i + rot - n_rr;
+                const uint8_t* slot = wait_full();
+                const int a = idx_in(hdr, C.ttok[ti][0], 0, S, 615);
+                const uint4* st = stage + (size_t)ti * cpt;
+                uint4 hrr[ND][NSUB];
+#pragma unroll
+                for (int i2 = 0; i2 < ND; ++i2)
+#pragma unroll
+                    for (int sb = 0; sb < NSUB; ++sb) hrr[i2][sb] = st[sb * nch_dn + lane + 32 * i2];
+                const float shv = C.rsh[ti];
                 int csl = 0;  // the code sum, for the offset-binary correction
 #pragma unroll
                 for (int i = 0; i < ND; ++i)
@@ -1034,6 +1070,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     const int rl = q * kDecWarps + gw;
                     if (lane == 0 && rl < rr_rows) ys[a * RRW + rl] = __fmul_rn((float)D, __fmul_rn(sdr[q], shv));
                 }
+                if (n_done == 0 && ctid == 0) DEC_TRACE(22);
+                ++n_done;
             }
             named_sync(kDecBar, kDecCons);  // every y of this CTA's rows is in shared memory
             if (ctid == 0) DEC_TRACE(21);

@@ -30,6 +30,15 @@ static bool dev_facts(DevFacts* out) {
     return true;
 }
 
+// Tokens the kernel instance for T tokens is compiled for (its shared control
+// block is sized for them).
+static size_t ctl_bytes(int T) {
+    if (T <= 1) return sizeof(DecCtl<1>);
+    if (T <= 2) return sizeof(DecCtl<2>);
+    if (T <= 4) return sizeof(DecCtl<4>);
+    return sizeof(DecCtl<8>);
+}
+
 bool decode_plan(const Dims& m, DecPlan* pl) {
     if (m.T < 1 || m.T > kDecMaxT || m.k > kDecMaxK) return false;
     DevFacts df;
@@ -49,27 +58,37 @@ bool decode_plan(const Dims& m, DecPlan* pl) {
     q.slot_bytes = slot;
     q.nu_gu = (m.f + kDecWarps - 1) / kDecWarps;
     q.nu_dn = (m.d + q.rd - 1) / q.rd;
-    const int ctl = (int)align_up(sizeof(DecCtl), 128);
+    const int ctl = (int)align_up(ctl_bytes(m.T), 128);
     const int xs = (int)align_up((size_t)m.T * m.d, 128);
     q.hs_grp_bytes = (int)align_up((size_t)m.T * m.f, 128);
-    // h staging of both consumer groups; the same bytes serve the top-k scratch
-    const int hs = (int)align_up(std::max((size_t)kDecGroups * q.hs_grp_bytes, (size_t)8 * m.T * m.E), 128);
-    const int room = optin - ctl - xs - hs - 1024;  // keep 1 KB for static shared memory
+    // single-token down by output-row ranges: every CTA's rows (whole quads)
+    // of one task fit a unit with f bytes to spare (the set of shapes this
+    // path has been measured and tested on), and the consumers stage every
+    // task's codes at once
+    const int sms = df.sms;
+    const int rr_rows_max = sms > 0 ? (m.d / 4 + sms - 1) / sms * 4 : 1 << 30;
+    const bool rr_shape = m.T == 1 && m.k + m.has_shared <= kDecRRMaxTasks && m.d % 4 == 0 && m.f % 16 == 0 &&
+                          m.S * (m.f / 16) <= kDecRRChunks * kDecCons && q.rd == kDecNQ * kDecWarps &&
+                          rr_rows_max <= kDecRRMaxRows && rr_rows_max * rb_dn <= wbytes - m.f;
+    // h staging of both consumer groups (the same bytes serve the top-k
+    // scratch); on the row-range path the codes of every task, then the
+    // per-row outputs of every assignment
+    const size_t hs_base = std::max((size_t)kDecGroups * q.hs_grp_bytes, (size_t)8 * m.T * m.E);
+    const size_t hs_rr = std::max(hs_base, (size_t)m.S * m.f + (size_t)m.S * kDecNQ * kDecWarps * 4);
     // an even slot count: the two consumer groups take alternate units, so
     // each group then owns the slots of its parity and waits on consecutive
     // phases of each (an odd count would let a group reach a slot two rounds
     // ahead, where a parity wait cannot tell the phases apart)
-    q.nslot = std::min(kDecMaxSlots, room / slot) / 2 * 2;
+    auto slots_for = [&](size_t hs) {
+        const int room = optin - ctl - xs - (int)align_up(hs, 128) - 1024;  // keep 1 KB for static shared memory
+        return std::min(kDecMaxSlots, room / slot) / 2 * 2;
+    };
+    // the row-range path only where it keeps the full ring
+    q.rowrange = rr_shape && slots_for(hs_rr) == kDecMaxSlots;
+    const int hs = (int)align_up(q.rowrange ? hs_rr : hs_base, 128);
+    q.nslot = slots_for((size_t)hs);
     if (q.nslot < 2) return false;
-    // single-token down by output-row ranges: every CTA's rows (whole quads)
-    // of one task fit a unit with f bytes to spare (the set of shapes this
-    // path has been measured and tested on), and the per-row outputs of all
-    // assignments fit the h staging area
-    const int sms = df.sms;
-    const int rr_rows_max = sms > 0 ? (m.d / 4 + sms - 1) / sms * 4 : 1 << 30;
-    q.rowrange = m.T == 1 && m.k + m.has_shared <= kDecRRMaxTasks && m.d % 4 == 0 &&
-                 q.rd == kDecNQ * kDecWarps && rr_rows_max <= kDecRRMaxRows &&
-                 rr_rows_max * rb_dn <= wbytes - m.f && (size_t)m.S * kDecNQ * kDecWarps * 4 <= (size_t)hs;
+    q.dn_rot = 1;
     q.xs_off = ctl;
     q.hs_off = ctl + xs;
     q.ring_off = ctl + xs + hs;

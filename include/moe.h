@@ -193,10 +193,11 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *         totals: [9] consumer wait for data, [10] producer wait for slots;
  *         producer: [12] rows known before routing issued, [13] routing
  *         received, [14] all rows issued, [15] all copies landed; one-token
- *         row-range down: [16] the CTA's designated task's h row complete (polled),
- *         [17] its codes and scale written, [20] first down unit's codes
- *         seen, [21] last down unit done.  Untouched entries are left as
- *         is. */
+ *         row-range down: [7] the CTA's designated tasks requantised, [16]
+ *         its first designated task's h row complete (polled), [17] its
+ *         codes and scale written, [20] every task's codes staged, [22] the
+ *         first down unit done, [21] the last.  Untouched entries are left
+ *         as is. */
 enum { MOE_PATH_AUTO = 0, MOE_PATH_MULTI = 1, MOE_PATH_DECODE = 2, MOE_PATH_TC = 3 };
 typedef struct {
     void* events[4];
