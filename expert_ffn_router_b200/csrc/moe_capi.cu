@@ -144,8 +144,13 @@ static int pick_ch(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8; }
 static Dims layout_dims(const moe_config* c, size_t ws_bytes);
 
 // Default of moe_config.tc_min_tokens: calls with at least this many tokens
-// run the experts on the tensor-core path.
-constexpr int kTcDefaultMinTokens = 16;
+// run the experts on the tensor-core path.  Measured on B200 at the GLM-5.2
+// expert shape (one layer, 256 experts, top-8, int4; us per call, decode
+// kernel vs tensor-core path): T = 1: 68 vs 136, T = 2: 137 vs 168, T = 3:
+// 222 vs 214, T = 4: 301 vs 251, T = 8: 878 vs 364 -- the decode kernel's ring
+// holds only two slots from three tokens on, while the tensor-core path keeps
+// its weight tiles flowing.
+constexpr int kTcDefaultMinTokens = 3;
 
 static bool use_tc(const moe_config* c, int T) {
     const int thr = c->tc_min_tokens == 0 ? kTcDefaultMinTokens : c->tc_min_tokens;
@@ -495,7 +500,10 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     if (path != MOE_PATH_AUTO && path != MOE_PATH_MULTI && path != MOE_PATH_DECODE && path != MOE_PATH_TC)
         return fail(MOE_EINVAL, "opts->path must be MOE_PATH_AUTO, MOE_PATH_MULTI, MOE_PATH_DECODE or MOE_PATH_TC");
     DecPlan pl{};
-    const bool dec_ok = (path == MOE_PATH_AUTO || path == MOE_PATH_DECODE) && decode_plan(m, &pl);
+    // AUTO: the tensor-core path from tc_min_tokens tokens on, else the
+    // single-launch decode kernel where the shape fits it, else MULTI
+    const bool auto_tc = path == MOE_PATH_AUTO && use_tc(cfg, T);
+    const bool dec_ok = ((path == MOE_PATH_AUTO && !auto_tc) || path == MOE_PATH_DECODE) && decode_plan(m, &pl);
     // the h-skip hook acts only where the hand-off polls values (one token,
     // row-range down); elsewhere it would give wrong output instead of a timeout
     if (!(dec_ok && pl.rowrange)) p.skip_h_task = -1;
@@ -512,7 +520,7 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         }
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (decode)");
     }
-    if (path == MOE_PATH_TC || (path == MOE_PATH_AUTO && use_tc(cfg, T))) {
+    if (path == MOE_PATH_TC || auto_tc) {
         Params q = base_params(cfg, m, ws, ws_bytes, true);
         q.pool = p.pool;
         q.scales = p.scales;

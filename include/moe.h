@@ -75,9 +75,10 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  *  routed blobs; wbits: 4 or 2; routed_scale: factor on the renormalised
  *  routed weights (2.5 for GLM-5.2).
  *  tc_min_tokens: calls of at least this many tokens run the experts on the
- *  int8 tensor-core (tcgen05) path (moe_layer with MOE_PATH_AUTO once the
- *  single-launch decode path does not apply, moe_expert_ffn, moe_expert_down);
- *  0 = library default (16), < 0 = never.
+ *  int8 tensor-core (tcgen05) path (moe_layer with MOE_PATH_AUTO,
+ *  moe_expert_ffn, moe_expert_down); 0 = library default (3: on B200 at the
+ *  GLM-5.2 expert shape the single-launch decode kernel is faster for one and
+ *  two tokens, the tensor-core path from three on), < 0 = never.
  * Limits (MOE_EINVAL otherwise): 1 <= k <= min(E, 32); E <= 1024;
  * d * wbits / 8 and f * wbits / 8 multiples of 16; d <= 8192; f <= 8192. */
 typedef struct {
@@ -179,8 +180,8 @@ MOE_API moe_status moe_layer(const moe_config* cfg, const moe_pool* pool, const 
  *        persistent kernel for T <= 8; MOE_EINVAL if the shape does not fit
  *        it) or MOE_PATH_TC (3: routing, then gate/up and down as int8
  *        grouped GEMMs on the tensor cores, tasks of up to 64 tokens per
- *        expert, then the combine).  AUTO takes DECODE where it fits, else TC
- *        when T >= tc_min_tokens, else MULTI.
+ *        expert, then the combine).  AUTO takes TC when T >= tc_min_tokens
+ *        (and the shape fits it), else DECODE where it fits, else MULTI.
  *  path_ran: set to the path that ran (MOE_PATH_DECODE, _MULTI or _TC).
  *  n_launches: set to the number of kernels the call launched.
  *  trace: optional DEVICE buffer of (number of SMs) x 32 uint64 that the

@@ -31,7 +31,13 @@ SMALL = {
                                             wbits=2),
     "wide_k": W.workload(0).replace(name="wide_k", d=256, f=96, n_experts=64, top_k=32, T=7),
 }
-PATHS = {"auto": M.MOE_PATH_AUTO, "multi": M.MOE_PATH_MULTI}
+PATHS = {"auto": M.MOE_PATH_AUTO, "multi": M.MOE_PATH_MULTI, "decode": M.MOE_PATH_DECODE}
+
+
+def auto_path(T):
+    """The path MOE_PATH_AUTO takes for T tokens with the default
+    tc_min_tokens (3) on shapes that fit both kernels."""
+    return M.MOE_PATH_DECODE if T <= 2 else M.MOE_PATH_TC
 
 # One-token decode on small pools of d = 2048 (the decode kernel's runtime-loop
 # rows): int4 and int2 rows, no shared expert, E > 256 (its shared-memory
@@ -171,7 +177,9 @@ def run_layer_gpu(wl, dl, x, accumulate_into=None, path="auto", ws=None):
     M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x), out, ws, accumulate=accumulate_into is not None,
                 topk_idx_out=idx, topk_w_out=w, opts=opts)
     assert_ok(ws)
-    if path == "auto" and T <= 8:
+    if path == "auto":
+        assert opts.path_ran == auto_path(T)
+    if path == "decode":
         assert opts.n_launches == 1 and opts.path_ran == M.MOE_PATH_DECODE  # the single-launch kernel ran
     if path == "multi":
         assert opts.path_ran == M.MOE_PATH_MULTI
@@ -198,6 +206,8 @@ def compare_layer(wl, L, x, out, g_idx, tokens=None):
 @pytest.mark.parametrize("name", list(SMALL))
 def test_layer_small(name, path):
     wl = SMALL[name]
+    if path == "decode" and wl.T > 8:
+        pytest.skip("the decode kernel takes at most 8 tokens")
     L = W.layer(wl, 0, 0)
     dl = W.device_layer(wl, 0, 0, host=L)
     x = x_host(wl)
@@ -211,7 +221,8 @@ def test_layer_small(name, path):
 
 def test_layer_decode_full_size():
     """The decode workload as the bench runs it: T = 1 per call, 8 token sets,
-    one workspace reused across calls; then T = 8, and the multi-kernel path."""
+    one workspace reused across calls; then T = 8 on the decode kernel and on
+    AUTO's tensor-core path, and the multi-kernel path."""
     wl = W.workload(1)
     L = W.layer(wl, 0, 0)
     dl = W.device_layer(wl, 0, 0, host=L)
@@ -223,7 +234,9 @@ def test_layer_decode_full_size():
         err, allowed = compare_layer(wl, L, x, out, g_idx)
         errs.append(err)
     x = x_host(wl, 20, 8)
-    out, g_idx, _ = run_layer_gpu(wl, dl, x, ws=ws)
+    out, g_idx, _ = run_layer_gpu(wl, dl, x, path="decode", ws=ws)
+    errs.append(compare_layer(wl, L, x, out, g_idx)[0])
+    out, g_idx, _ = run_layer_gpu(wl, dl, x, ws=ws)  # AUTO: the tensor-core path at 8 tokens
     errs.append(compare_layer(wl, L, x, out, g_idx)[0])
     out, g_idx, _ = run_layer_gpu(wl, dl, x_host(wl, 0), path="multi", ws=ws)
     errs.append(compare_layer(wl, L, x_host(wl, 0), out, g_idx)[0])

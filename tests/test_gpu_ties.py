@@ -116,6 +116,8 @@ LAYER_CASES = [  # (kind, E, k, T, path)
     ("dup", 512, 8, 1, "auto"), ("zero", 512, 8, 5, "auto"), ("dup", 1024, 32, 1, "auto"),
     ("dup", 1024, 32, 8, "auto"), ("dup", 512, 8, 32, "auto"), ("dup", 1024, 32, 32, "auto"),
     ("zero", 1024, 32, 12, "multi"), ("dup", 512, 8, 6, "multi"), ("dup", 256, 8, 24, "multi"),
+    ("dup", 8, 2, 6, "decode"), ("zero", 256, 8, 8, "decode"), ("zero", 512, 8, 5, "decode"),
+    ("dup", 1024, 32, 8, "decode"),
 ]
 
 
@@ -125,7 +127,7 @@ def test_layer_exact_ties_and_wide_pools(kind, E, k, T, path):
     oracle (no allowance) and the output within the layer tolerance.  E = 512
     and 1024 run the decode kernel's shared-memory top-k (T <= 8), the tiled
     router's top-k with the separate bucketing kernel and the tensor-core path
-    (T >= 16), and the dp4a multi-kernel path."""
+    (AUTO from 3 tokens on), and the dp4a multi-kernel path."""
     wl = W.workload(0).replace(name=f"ties_{kind}_E{E}", d=256, f=128, n_experts=E, top_k=k, T=T)
     wr, bias = tie_router(E, wl.d, k, kind)
     L = W.layer(wl, 0, 0)
@@ -138,11 +140,12 @@ def test_layer_exact_ties_and_wide_pools(kind, E, k, T, path):
     idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
     w = torch.zeros(T, k, device="cuda")
     opts = M.MoeLayerOpts()
-    opts.path = {"auto": M.MOE_PATH_AUTO, "multi": M.MOE_PATH_MULTI}[path]
+    opts.path = {"auto": M.MOE_PATH_AUTO, "multi": M.MOE_PATH_MULTI, "decode": M.MOE_PATH_DECODE}[path]
     M.moe_layer(cfg, M.make_pool(dl.pool_w, dl.pool_s), dl.w_router, dl.bias, x.cuda(), out, ws,
                 topk_idx_out=idx, topk_w_out=w, opts=opts)
     assert M.moe_poll_status(ws) == M.MOE_OK
-    expect = {"multi": M.MOE_PATH_MULTI}.get(path, M.MOE_PATH_DECODE if T <= 8 else M.MOE_PATH_TC)
+    expect = {"multi": M.MOE_PATH_MULTI, "decode": M.MOE_PATH_DECODE}.get(
+        path, M.MOE_PATH_DECODE if T <= 2 else M.MOE_PATH_TC)
     assert opts.path_ran == expect
     r = O.workload_layer(wl, 0, 0, x, L=L)
     _, _, o_sel = oracle_route(x, wr, bias, k)
