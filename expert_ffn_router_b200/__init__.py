@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe_bounds.so" if os.environ.get("MOE_LIBRARY"
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "moe.h")
 
 MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_ENOSPACE, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE = 0, -1, -2, -3, -4, -5, -6
+MOE_IO_X_HOST, MOE_IO_OUT_HOST = 1, 2  # moe_layer_opts.io_host bits
 MOE_F32, MOE_BF16 = 0, 1
 MOE_PATH_AUTO, MOE_PATH_MULTI, MOE_PATH_DECODE, MOE_PATH_TC = 0, 1, 2, 3
 
@@ -54,7 +55,7 @@ class MoeConfig(ctypes.Structure):
 class MoeLayerOpts(ctypes.Structure):
     _fields_ = [("events", ctypes.c_void_p * 4), ("path", ctypes.c_int32), ("n_launches", ctypes.c_int32),
                 ("trace", ctypes.c_void_p), ("path_ran", ctypes.c_int32),
-                ("wait_limit_us", ctypes.c_int32), ("test_skip_h", ctypes.c_int32)]
+                ("wait_limit_us", ctypes.c_int32), ("test_skip_h", ctypes.c_int32), ("io_host", ctypes.c_int32)]
 
 
 class MoePool(ctypes.Structure):
@@ -114,10 +115,14 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> int:
     return s.cuda_stream
 
 
-def _ptr(t: Optional[torch.Tensor], dtype=None, numel: Optional[int] = None, name: str = "") -> Optional[int]:
+def _ptr(t: Optional[torch.Tensor], dtype=None, numel: Optional[int] = None, name: str = "",
+         host: bool = False) -> Optional[int]:
     if t is None:
         return None
-    if not t.is_cuda:
+    if host:
+        if t.is_cuda or not t.is_pinned():
+            raise ValueError(f"{name}: expected a pinned host tensor")
+    elif not t.is_cuda:
         raise ValueError(f"{name}: expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous tensor")
@@ -227,10 +232,12 @@ def moe_layer(cfg: MoeConfig, pool: MoePool, w_router: torch.Tensor, bias: torch
               topk_w_out=None, stream=None, opts: Optional[MoeLayerOpts] = None):
     """moe_layer, or moe_layer_ex when ``opts`` is given."""
     T = x.shape[0]
+    io = opts.io_host if opts is not None else 0
     args = (ctypes.byref(cfg), ctypes.byref(pool),
             _ptr(w_router, torch.float32, cfg.n_experts * cfg.d, "w_router"),
-            _ptr(bias, torch.float32, cfg.n_experts, "bias"), _ptr(x, name="x"), _xdtype(x), T,
-            _ptr(out, torch.float32, T * cfg.d, "out"), 1 if accumulate else 0,
+            _ptr(bias, torch.float32, cfg.n_experts, "bias"), _ptr(x, name="x", host=bool(io & MOE_IO_X_HOST)),
+            _xdtype(x), T,
+            _ptr(out, torch.float32, T * cfg.d, "out", host=bool(io & MOE_IO_OUT_HOST)), 1 if accumulate else 0,
             _ptr(topk_idx_out, torch.int32, T * cfg.top_k, "topk_idx_out"),
             _ptr(topk_w_out, torch.float32, T * cfg.top_k, "topk_w_out"),
             _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream))

@@ -453,6 +453,28 @@ moe_status moe_expert_down(const moe_config* cfg, const moe_pool* pool, int32_t 
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_down");
 }
 
+// The device-side address of pinned host memory (MOE_EINVAL if p is not host
+// memory the device can address).
+static moe_status host_mapped(const void* p, const char* name, const void** dev) {
+    cudaPointerAttributes a{};
+    const cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) return cuda_fail(e, (std::string(name) + ": cudaPointerGetAttributes").c_str());
+    if (a.type != cudaMemoryTypeHost || !a.devicePointer)
+        return fail(MOE_EINVAL, std::string(name) + ": not pinned host memory mapped into the device's address space");
+    if (!aligned16(a.devicePointer)) return fail(MOE_EALIGN, std::string(name) + " is not 16-byte aligned");
+    *dev = a.devicePointer;
+    return MOE_OK;
+}
+
+// Copy `bytes` (a multiple of 16) from mapped host memory into device memory.
+static cudaError_t launch_stage_in(const void* src, void* dst, size_t bytes, cudaStream_t s) {
+    const long long n16 = (long long)(bytes / 16);
+    const long long per_cta = 4ll * kThreads;  // four chunks in flight per thread
+    const int grid = (int)std::max(1ll, std::min((n16 + per_cta - 1) / per_cta, 4ll * 148));
+    k_stage_in<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16);
+    return cudaGetLastError();
+}
+
 moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float* w_router, const float* bias,
                         const void* x, moe_dtype dtype, int32_t T, float* out, int32_t accumulate,
                         int32_t* topk_idx_out, float* topk_w_out, void* ws, size_t ws_bytes, moe_stream_t stream,
@@ -466,7 +488,10 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         opts->path_ran = MOE_PATH_AUTO;
         if (opts->wait_limit_us < 0 || opts->test_skip_h < 0)
             return fail(MOE_EINVAL, "opts->wait_limit_us and opts->test_skip_h must be >= 0");
+        if (opts->io_host & ~(MOE_IO_X_HOST | MOE_IO_OUT_HOST))
+            return fail(MOE_EINVAL, "opts->io_host: unknown bits");
     }
+    const int io = opts ? opts->io_host : 0;
     if (T == 0) return MOE_OK;
     MOE_TRY(check_ptr(pool->w, "pool->w"));
     MOE_TRY(check_ptr(pool->s, "pool->s"));
@@ -474,6 +499,14 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     MOE_TRY(check_ptr(bias, "bias"));
     MOE_TRY(check_ptr(x, "x"));
     MOE_TRY(check_ptr(out, "out"));
+    // the device-side addresses of host buffers (their own, with unified addressing)
+    const void* x_host = nullptr;
+    if (io & MOE_IO_X_HOST) MOE_TRY(host_mapped(x, "x", &x_host));
+    if (io & MOE_IO_OUT_HOST) {
+        const void* o = nullptr;
+        MOE_TRY(host_mapped(out, "out", &o));
+        out = static_cast<float*>(const_cast<void*>(o));
+    }
     MOE_TRY(check_ptr(topk_idx_out, "topk_idx_out", true));
     MOE_TRY(check_ptr(topk_w_out, "topk_w_out", true));
     const Dims m = dims_of(cfg, T, cfg->top_k + cfg->has_shared);
@@ -510,12 +543,16 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     if (path == MOE_PATH_DECODE && !dec_ok) return fail(MOE_EINVAL, "shape does not fit the single-launch decode path");
     if (path == MOE_PATH_TC && !tc_shape_ok(m)) return fail(MOE_EINVAL, "shape does not fit the tensor-core path");
     cudaError_t e = mark(0);
+    if (e == cudaSuccess && x_host) {  // one read of x over the host link, into the workspace
+        e = launch_stage_in(x_host, p.ws.xin, (size_t)T * cfg->d * (dtype == MOE_BF16 ? 2 : 4), s);
+        x = p.ws.xin;
+    }
     if (dec_ok) {
         if (e == cudaSuccess)
             e = launch_decode(p, pl, x, dtype == MOE_BF16, s);
         if (e == cudaSuccess) e = mark(3);  // [1] and [2] fall inside the one kernel: not recorded
         if (opts) {
-            opts->n_launches = 1;
+            opts->n_launches = 1 + (x_host ? 1 : 0);
             opts->path_ran = MOE_PATH_DECODE;
         }
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (decode)");
@@ -540,7 +577,7 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         if (e == cudaSuccess) e = launch_combine(q, s);
         if (e == cudaSuccess) e = mark(3);
         if (opts) {
-            opts->n_launches = (T <= 8 ? 1 : cfg->n_experts <= 256 ? 3 : 4) + 5;
+            opts->n_launches = (T <= 8 ? 1 : cfg->n_experts <= 256 ? 3 : 4) + 5 + (x_host ? 1 : 0);
             opts->path_ran = MOE_PATH_TC;
         }
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer (tensor cores)");
@@ -552,7 +589,7 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     if (e == cudaSuccess) e = launch_down(p, tl, false, s);
     if (e == cudaSuccess) e = mark(3);
     if (opts) {
-        opts->n_launches = (T <= 8 ? 1 : cfg->n_experts <= 256 ? 3 : 4) + 2;
+        opts->n_launches = (T <= 8 ? 1 : cfg->n_experts <= 256 ? 3 : 4) + 2 + (x_host ? 1 : 0);
         opts->path_ran = MOE_PATH_MULTI;
     }
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer");

@@ -66,6 +66,7 @@ struct Ws {
     int32_t* hcs;      // [T*S]      sum of the hq codes of each assignment (tensor-core down)
     uint8_t* xb;       // tensor-core operand B of gate/up: per task, activation rows in MMA layout
     uint8_t* hb;       // tensor-core operand B of down: per task, hq rows in MMA layout
+    uint8_t* xin;      // [T][d] x as given (<= 4 bytes per value), copied in from host memory
     size_t bytes;
 };
 
@@ -129,6 +130,7 @@ inline Ws ws_carve(const Dims& m, void* base) {
     w.hcs = (int32_t*)take(A * 4);
     w.xb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.d, m.wb));
     w.hb = (uint8_t*)take(tc_rows_bound(m) * tc_kpad(m.f, m.wb));
+    w.xin = (uint8_t*)take(T * m.d * 4);
     w.bytes = off;
     return w;
 }

@@ -41,6 +41,23 @@ __device__ void quantize_token(const XT* x, int d, int8_t* xq, float* sx, int32_
     }
 }
 
+// Copy n16 16-byte chunks from src -- pinned host memory mapped into the
+// device's address space -- to device memory, four independent loads in
+// flight per thread (plain coherent loads: no read-only-cache path on host
+// memory).
+__global__ void __launch_bounds__(kThreads) k_stage_in(const uint4* src, uint4* dst, long long n16) {
+    const long long stride = (long long)gridDim.x * kThreads;
+    long long i = (long long)blockIdx.x * kThreads + threadIdx.x;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        const uint4 a = src[i], b = src[i + stride], c = src[i + 2 * stride], e = src[i + 3 * stride];
+        dst[i] = a;
+        dst[i + stride] = b;
+        dst[i + 2 * stride] = c;
+        dst[i + 3 * stride] = e;
+    }
+    for (; i < n16; i += stride) dst[i] = src[i];
+}
+
 template <typename XT>
 __global__ void __launch_bounds__(kThreads) k_quantize(const XT* __restrict__ x, int T, int d,
                                                         int8_t* __restrict__ xq, float* __restrict__ sx,

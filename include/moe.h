@@ -218,7 +218,17 @@ typedef struct {
      * routed experts in ascending id order), so that every wait on them runs
      * out; ignored on every other path; 0 = off. */
     int32_t test_skip_h;
+    /* in: where x and out live.  MOE_IO_X_HOST: x is pinned host memory
+     * mapped into the device's address space (cudaHostAlloc, or
+     * cudaHostRegister with mapping; with unified addressing the host pointer
+     * is the device pointer); the call first copies it into the workspace with
+     * a small kernel (one read over the host link, no DMA copy), then runs
+     * the layer on the copy.  MOE_IO_OUT_HOST: out is such memory; the
+     * kernels write (and in accumulate mode read) it directly.  0 = both in
+     * device memory. */
+    int32_t io_host;
 } moe_layer_opts;
+enum { MOE_IO_X_HOST = 1, MOE_IO_OUT_HOST = 2 };
 
 /* moe_layer with options (opts may be NULL, then identical to moe_layer). */
 MOE_API moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float* w_router,

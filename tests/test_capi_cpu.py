@@ -109,3 +109,7 @@ def test_layer_opts_rejects_negative_test_fields():
     st = L.moe_layer_ex(ctypes.byref(c), ctypes.byref(pool), FAKE, FAKE, FAKE, 0, 4, FAKE, 0, None, None, FAKE,
                         1 << 40, None, ctypes.byref(o))
     assert st == M.MOE_EINVAL
+    o.test_skip_h, o.io_host = 0, 4  # an unknown io_host bit
+    st = L.moe_layer_ex(ctypes.byref(c), ctypes.byref(pool), FAKE, FAKE, FAKE, 0, 4, FAKE, 0, None, None, FAKE,
+                        1 << 40, None, ctypes.byref(o))
+    assert st == M.MOE_EINVAL
