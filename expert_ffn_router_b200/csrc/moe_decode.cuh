@@ -74,6 +74,7 @@ struct DecPlan {
     int hs_grp_bytes;  // h staging bytes of one consumer group (T * f)
     int rowrange;      // single-token down by output-row ranges (see step 6r)
     int dn_rot;        // row-range: CTA c takes the down tasks from task c mod n_tasks on
+    int gu_rmaj;       // row-range: routed gate/up units ordered row block first, tasks inner
 };
 // Row-range down unit (single token): [rows x down row][row scales at wbytes].
 constexpr int kDecRRMaxRows = 44;
@@ -342,6 +343,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     const int rr_lo = (int)((long long)c * (d / 4) / G) * 4;
     const int rr_rows = (int)((long long)(c + 1) * (d / 4) / G) * 4 - rr_lo;
     const bool rowrange = TM == 1 && ND > 0 && pl.rowrange;
+    // every CTA takes an equal share of every routed expert's rows (experts
+    // stream at different speeds, and a CTA's finish time is then the average)
+    const bool rmaj = rowrange && pl.gu_rmaj;
     if (tid == 0) DEC_TRACE(0);
     const int n_my_router = c < E ? (E - c + G - 1) / G : 0;  // experts c, c+G, ...
     const int n_router_units = (n_my_router + pl.rr - 1) / pl.rr;
@@ -414,14 +418,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
                 const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
                 n_units = hi - lo;
-                ti = HS + (int)(lo / pl.nu_gu);
-                j = (int)(lo % pl.nu_gu);
+                if (rmaj) {  // unit g: row block g / n_routed of task HS + g mod n_routed
+                    ti = HS + (int)(lo % (n_tasks - HS));
+                    j = (int)(lo / (n_tasks - HS));
+                } else {
+                    ti = HS + (int)(lo / pl.nu_gu);
+                    j = (int)(lo % pl.nu_gu);
+                }
                 jstep = 1;
                 jwrap = pl.nu_gu;
                 sh_blob = -1;
             }
+            const bool tasks_inner = ph == 1 && rmaj;
             for (long long g = 0; g < n_units; ++g) {
                 issue_gu(sh_blob >= 0 ? sh_blob : C.tasks[ti].x, j);
+                if (tasks_inner) {
+                    if (++ti == n_tasks) {
+                        ti = HS;
+                        ++j;
+                    }
+                    continue;
+                }
                 j += jstep;
                 if (j == jwrap) {
                     j = 0;
@@ -899,13 +916,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             const long long Nr = (long long)(n_tasks - HS) * pl.nu_gu;
             const long long lo = c * Nr / G, hi = (c + 1) * Nr / G;
             n_units = hi - lo;
-            ti = HS + (int)(lo / pl.nu_gu);
-            j = (int)(lo % pl.nu_gu);
+            if (rmaj) {  // the producer's order: row block first, tasks inner
+                ti = HS + (int)(lo % (n_tasks - HS));
+                j = (int)(lo / (n_tasks - HS));
+            } else {
+                ti = HS + (int)(lo / pl.nu_gu);
+                j = (int)(lo % pl.nu_gu);
+            }
             jstep = 1;
             jwrap = pl.nu_gu;
         }
+        const bool tasks_inner = ph == 2 && rmaj;
         for (long long g = 0; g < n_units; ++g, next_unit()) {
             if (mine()) gu_unit(ti, j);
+            if (tasks_inner) {
+                if (++ti == n_tasks) {
+                    ti = HS;
+                    ++j;
+                }
+                continue;
+            }
             j += jstep;
             if (j == jwrap) {
                 j = 0;

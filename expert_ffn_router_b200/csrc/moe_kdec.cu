@@ -89,6 +89,7 @@ bool decode_plan(const Dims& m, DecPlan* pl) {
     q.nslot = slots_for((size_t)hs);
     if (q.nslot < 2) return false;
     q.dn_rot = 1;
+    q.gu_rmaj = 1;
     q.xs_off = ctl;
     q.hs_off = ctl + xs;
     q.ring_off = ctl + xs + hs;
