@@ -40,13 +40,16 @@ def lib():
         L.oracle_pack.argtypes = [_I, _P, _I64, _P]
         L.oracle_quantize.argtypes = [_P, _I, _I, _P, _P]
         L.oracle_route.argtypes = [_P, _I, _I, _I, _I, _P, _P, _D, _P, _P, _P, _P, _P]
+        L.oracle_route_p.argtypes = [_P, _I, _I, _I, _I, _P, _P, _D, ctypes.c_float, _P, _P, _P, _P, _P]
         L.oracle_down.argtypes = [_I, _I, _I, _P, _P, _P, _P, _I, _P, _P]
         L.oracle_expert.argtypes = [_I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P]
         L.oracle_layer.argtypes = [_I, _I, _I, _I, _I, _I, _D, _P, _P, _P, _P, _P, _I, _P, _P, _P,
                                    _P, _P]
+        L.oracle_layer_p.argtypes = [_I, _I, _I, _I, _I, _I, _D, ctypes.c_float, _P, _P, _P, _P, _P, _I, _P,
+                                     _P, _P, _P, _P]
         L.oracle_rmsnorm.argtypes = [_P, _I, _I, _D, _P]
-        for fn in ("oracle_unpack", "oracle_pack", "oracle_quantize", "oracle_route", "oracle_down",
-                   "oracle_expert", "oracle_layer", "oracle_rmsnorm"):
+        for fn in ("oracle_unpack", "oracle_pack", "oracle_quantize", "oracle_route", "oracle_route_p",
+                   "oracle_down", "oracle_expert", "oracle_layer", "oracle_layer_p", "oracle_rmsnorm"):
             getattr(L, fn).restype = _I
         _lib = L
     return _lib
@@ -104,8 +107,9 @@ def quantize(x) -> Tuple[np.ndarray, np.ndarray]:
     return q, s
 
 
-def route(x, w_router, bias, k: int, routed_scale: float = 2.5, want_scores: bool = False):
-    """Returns idx int32 [T][k], w float64 [T][k] (and logits, s, sel fp32 [T][E])."""
+def route(x, w_router, bias, k: int, routed_scale: float = 2.5, want_scores: bool = False, topp: float = 0.0):
+    """Returns idx int32 [T][k], w float64 [T][k] (and logits, s, sel fp32 [T][E]).
+    topp in (0, 1): TOPP truncation (oracle.c, a1'): dropped slots idx -1, w 0."""
     x = _np(x, np.float32)
     wr = _np(w_router, np.float32)
     b = _np(bias, np.float32)
@@ -116,8 +120,8 @@ def route(x, w_router, bias, k: int, routed_scale: float = 2.5, want_scores: boo
     lg = np.empty((T, E), np.float32) if want_scores else None
     s = np.empty((T, E), np.float32) if want_scores else None
     sel = np.empty((T, E), np.float32) if want_scores else None
-    _check(lib().oracle_route(_ptr(x), T, d, E, k, _ptr(wr), _ptr(b), routed_scale, _ptr(idx),
-                              _ptr(w), _ptr(lg), _ptr(s), _ptr(sel)), "oracle_route")
+    _check(lib().oracle_route_p(_ptr(x), T, d, E, k, _ptr(wr), _ptr(b), routed_scale, topp, _ptr(idx),
+                                _ptr(w), _ptr(lg), _ptr(s), _ptr(sel)), "oracle_route_p")
     if want_scores:
         return idx, w, lg, s, sel
     return idx, w
@@ -153,7 +157,7 @@ def down(d: int, f: int, wbits: int, blob, scales, hq, sh) -> Dict[str, np.ndarr
 
 def layer(d: int, f: int, E: int, k: int, has_shared: int, wbits: int, routed_scale: float,
           blobs: Sequence[Optional[np.ndarray]], scales: Sequence[Optional[np.ndarray]], w_router,
-          bias, x) -> Dict[str, np.ndarray]:
+          bias, x, topp: float = 0.0) -> Dict[str, np.ndarray]:
     """Full layer on x fp32 [T][d].  blobs/scales: per-expert arrays (shared last);
     entries may be None for experts no token selects."""
     x = _np(x, np.float32)
@@ -171,9 +175,9 @@ def layer(d: int, f: int, E: int, k: int, has_shared: int, wbits: int, routed_sc
     w = np.empty((T, k), np.float64)
     xq = np.empty((T, d), np.int8)
     sx = np.empty(T, np.float32)
-    _check(lib().oracle_layer(d, f, E, k, has_shared, wbits, routed_scale, ctypes.cast(bt, _P),
-                              ctypes.cast(st, _P), _ptr(wr), _ptr(b), _ptr(x), T, _ptr(out),
-                              _ptr(idx), _ptr(w), _ptr(xq), _ptr(sx)), "oracle_layer")
+    _check(lib().oracle_layer_p(d, f, E, k, has_shared, wbits, routed_scale, topp, ctypes.cast(bt, _P),
+                                ctypes.cast(st, _P), _ptr(wr), _ptr(b), _ptr(x), T, _ptr(out),
+                                _ptr(idx), _ptr(w), _ptr(xq), _ptr(sx)), "oracle_layer_p")
     return dict(out=out, idx=idx, w=w, xq=xq, sx=sx)
 
 
@@ -195,8 +199,9 @@ def workload_layer(wl, seed: int, layer_idx: int, x_in, L=None, blob_cache=None)
     if L is None:
         L = W.layer(wl, seed, layer_idx)
     x_in = _np(x_in, np.float32)
-    idx, _ = route(x_in, L.w_router, L.bias, wl.top_k, wl.routed_scale)
-    need = sorted(set(idx.reshape(-1).tolist()) | ({wl.n_experts} if wl.has_shared else set()))
+    topp = getattr(wl, "topp", 0.0)
+    idx, _ = route(x_in, L.w_router, L.bias, wl.top_k, wl.routed_scale, topp=topp)
+    need = sorted((set(idx.reshape(-1).tolist()) - {-1}) | ({wl.n_experts} if wl.has_shared else set()))
     blobs: List[Optional[np.ndarray]] = [None] * wl.n_blobs
     scales: List[Optional[np.ndarray]] = [None] * wl.n_blobs
     sc_all = L.scales.numpy()
@@ -210,7 +215,7 @@ def workload_layer(wl, seed: int, layer_idx: int, x_in, L=None, blob_cache=None)
                 blob_cache[key] = blobs[e]
         scales[e] = np.ascontiguousarray(sc_all[e])
     return layer(wl.d, wl.f, wl.n_experts, wl.top_k, wl.has_shared, wl.wbits, wl.routed_scale,
-                 blobs, scales, L.w_router, L.bias, x_in)
+                 blobs, scales, L.w_router, L.bias, x_in, topp=topp)
 
 
 def workload_stack(wl, seed: int, x0, n_layers: Optional[int] = None, eps: float = 1e-6,

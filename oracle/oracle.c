@@ -17,6 +17,12 @@
  *       by routed_scale.         [takumi3488 article, teacher-forcing section:
  *       "DeepSeek-V3 style router"; top-8 of 256 and top-2 of 8 from the coli
  *       info logs; no group-limited selection -- reading]
+ *   a1' TOPK/TOPP truncation (opt-in, p in (0, 1)): keep the smallest prefix of
+ *       the selected slots, in selection order, whose normalised scores sum to
+ *       at least p; the dropped slots select no expert; the kept weights are
+ *       renormalised over the kept scores.   [reading: agentlenshq benchmark
+ *       table, the `--topp 0.7` rows, and the TOPK / TOPP options of the
+ *       takumi3488 run logs; the pages give no definition]
  *   a3  gate/up: int32 dot products of packed int4 / int2 codes with the int8
  *       activation codes; dequantised by (per-row scale * s_x); h = SiLU(g)*u.
  *       [agentlenshq summary: packed int4/int2 with per-row scales and
@@ -131,12 +137,18 @@ int oracle_quantize(const float* x, int T, int d, int8_t* q, float* s) {
     return ORACLE_OK;
 }
 
-/* a1: router.  x fp32 [T][d], wr fp32 [E][d], bias fp32 [E].
+/* a1 (+ a1'): router.  x fp32 [T][d], wr fp32 [E][d], bias fp32 [E].
  * Outputs idx [T][k] (slot order = selection score descending, ties to the
- * lower expert index), w fp64 [T][k]; optional logits/scores/sel fp32 [T][E]. */
-int oracle_route(const float* x, int T, int d, int E, int k, const float* wr, const float* bias,
-                 double routed_scale, int32_t* idx, double* w, float* logits_out, float* s_out,
-                 float* sel_out) {
+ * lower expert index), w fp64 [T][k]; optional logits/scores/sel fp32 [T][E].
+ * topp in (0, 1) truncates (a1'): the decision, an integer, is taken in
+ * float32 in slot order -- S = the float sum of the k selected scores, thr =
+ * float(topp * S); slot j is kept iff j == 0 or the float sum of the scores of
+ * slots 0..j-1 is below thr -- and a dropped slot gets idx -1 and weight 0;
+ * the kept weights are the kept scores over their (float64) sum, times
+ * routed_scale.  Any other topp: no truncation. */
+int oracle_route_p(const float* x, int T, int d, int E, int k, const float* wr, const float* bias,
+                   double routed_scale, float topp, int32_t* idx, double* w, float* logits_out,
+                   float* s_out, float* sel_out) {
     if (!x || !wr || !bias || !idx || !w || T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E)
         return ORACLE_EINVAL;
     float* s = (float*)malloc(sizeof(float) * (size_t)E);
@@ -157,7 +169,7 @@ int oracle_route(const float* x, int T, int d, int E, int k, const float* wr, co
             if (s_out) s_out[(int64_t)t * E + e] = s[e];
             if (sel_out) sel_out[(int64_t)t * E + e] = sel[e];
         }
-        double sum = 0.0;
+        int32_t* it = idx + (int64_t)t * k;
         for (int j = 0; j < k; ++j) {
             int best = -1;
             for (int e = 0; e < E; ++e) {
@@ -165,14 +177,38 @@ int oracle_route(const float* x, int T, int d, int E, int k, const float* wr, co
                 if (best < 0 || sel[e] > sel[best]) best = e; /* strict: ties keep the lower index */
             }
             taken[best] = 1;
-            idx[(int64_t)t * k + j] = best;
-            sum += (double)s[best];
+            it[j] = best;
         }
-        for (int j = 0; j < k; ++j)
-            w[(int64_t)t * k + j] = (double)s[idx[(int64_t)t * k + j]] / sum * routed_scale;
+        int m = k; /* slots kept */
+        if (topp > 0.0f && topp < 1.0f) {
+            float S = 0.0f;
+            for (int j = 0; j < k; ++j) S = S + s[it[j]];
+            const float thr = topp * S;
+            float before = 0.0f; /* float sum of the scores of the slots before j */
+            for (int j = 0; j < k; ++j) {
+                if (j > 0 && !(before < thr)) { m = j; break; }
+                before = before + s[it[j]];
+            }
+        }
+        double sum = 0.0;
+        for (int j = 0; j < m; ++j) sum += (double)s[it[j]];
+        for (int j = 0; j < k; ++j) {
+            if (j < m) {
+                w[(int64_t)t * k + j] = (double)s[it[j]] / sum * routed_scale;
+            } else {
+                it[j] = -1;
+                w[(int64_t)t * k + j] = 0.0;
+            }
+        }
     }
     free(s); free(sel); free(taken);
     return ORACLE_OK;
+}
+
+int oracle_route(const float* x, int T, int d, int E, int k, const float* wr, const float* bias,
+                 double routed_scale, int32_t* idx, double* w, float* logits_out, float* s_out,
+                 float* sel_out) {
+    return oracle_route_p(x, T, d, E, k, wr, bias, routed_scale, 0.0f, idx, w, logits_out, s_out, sel_out);
 }
 
 /* int dot of one packed row (n codes) with n int8 activation codes, in int64. */
@@ -255,18 +291,19 @@ int oracle_expert(int d, int f, int wbits, const uint8_t* blob, const float* sc,
 /* Full layer.  blobs / scales: tables of n_experts + has_shared pointers
  * (entry n_experts = shared expert); an entry may be NULL if no token selects
  * that expert.  x fp32 [T][d].  Outputs: out fp64 [T][d], idx [T][k], w fp64
- * [T][k]; xq/sx (nullable) the quantised input. */
-int oracle_layer(int d, int f, int E, int k, int has_shared, int wbits, double routed_scale,
-                 const uint8_t* const* blobs, const float* const* scales, const float* wr,
-                 const float* bias, const float* x, int T, double* out, int32_t* idx, double* w,
-                 int8_t* xq_out, float* sx_out) {
+ * [T][k]; xq/sx (nullable) the quantised input.  topp as in oracle_route_p
+ * (a dropped slot contributes nothing). */
+int oracle_layer_p(int d, int f, int E, int k, int has_shared, int wbits, double routed_scale, float topp,
+                   const uint8_t* const* blobs, const float* const* scales, const float* wr,
+                   const float* bias, const float* x, int T, double* out, int32_t* idx, double* w,
+                   int8_t* xq_out, float* sx_out) {
     if (!blobs || !scales || !wr || !bias || !x || !out || !idx || !w || T < 0) return ORACLE_EINVAL;
     int8_t* xq = (int8_t*)malloc((size_t)T * (size_t)d + 1);
     float* sx = (float*)malloc(sizeof(float) * (size_t)T + 1);
     double* y = (double*)malloc(sizeof(double) * (size_t)d);
     if (!xq || !sx || !y) { free(xq); free(sx); free(y); return ORACLE_EINVAL; }
     int rc = oracle_quantize(x, T, d, xq, sx);
-    if (!rc) rc = oracle_route(x, T, d, E, k, wr, bias, routed_scale, idx, w, NULL, NULL, NULL);
+    if (!rc) rc = oracle_route_p(x, T, d, E, k, wr, bias, routed_scale, topp, idx, w, NULL, NULL, NULL);
     for (int t = 0; !rc && t < T; ++t) {
         double* o = out + (int64_t)t * d;
         for (int r = 0; r < d; ++r) o[r] = 0.0;
@@ -276,6 +313,7 @@ int oracle_layer(int d, int f, int E, int k, int has_shared, int wbits, double r
             if (j < k) { e = idx[(int64_t)t * k + j]; wt = w[(int64_t)t * k + j]; }
             else if (has_shared) { e = E; wt = 1.0; }
             else break;
+            if (e < 0) continue; /* a slot dropped by the truncation */
             if (!blobs[e] || !scales[e]) { rc = ORACLE_ENULL; break; }
             rc = oracle_expert(d, f, wbits, blobs[e], scales[e], xq + (int64_t)t * d, sx + t, 1,
                                NULL, NULL, NULL, NULL, NULL, y);
@@ -286,6 +324,14 @@ int oracle_layer(int d, int f, int E, int k, int has_shared, int wbits, double r
     if (!rc && sx_out) memcpy(sx_out, sx, sizeof(float) * (size_t)T);
     free(xq); free(sx); free(y);
     return rc;
+}
+
+int oracle_layer(int d, int f, int E, int k, int has_shared, int wbits, double routed_scale,
+                 const uint8_t* const* blobs, const float* const* scales, const float* wr,
+                 const float* bias, const float* x, int T, double* out, int32_t* idx, double* w,
+                 int8_t* xq_out, float* sx_out) {
+    return oracle_layer_p(d, f, E, k, has_shared, wbits, routed_scale, 0.0f, blobs, scales, wr, bias, x, T,
+                          out, idx, w, xq_out, sx_out);
 }
 
 /* Parameter-free RMSNorm of the residual stream (stacked workloads; reading):

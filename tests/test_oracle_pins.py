@@ -327,3 +327,82 @@ def test_rmsnorm_closed_forms():
     np.testing.assert_allclose(y[0], [3 / math.sqrt(9 + 1e-6)] * 8, rtol=1e-7)
     np.testing.assert_allclose(y[1], [-2 / math.sqrt(4 + 1e-6), 2 / math.sqrt(4 + 1e-6)] * 4, rtol=1e-7)
     assert (y[2] == 0).all()
+
+
+# --------------------------------------------------------------------------
+# a1' TOPK/TOPP truncation (opt-in): smallest prefix of the selected slots
+# whose normalised scores reach p, the rest dropped (idx -1, weight 0), the
+# kept weights renormalised
+# --------------------------------------------------------------------------
+def test_topp_hand_cases():
+    x, wr, _ = hand_router()
+    bias = np.zeros(4, np.float32)
+    # token 0: s = [1/2, 3/4, 1/4, 1/2] -> slots: experts 1, 0, 3, 2 with scores
+    # .75, .5, .5, .25 (sum 2): prefixes before each slot 0, .75, 1.25, 1.75
+    cases = {
+        0.3: ([1, -1, -1, -1], [2.5, 0, 0, 0]),                       # thr .6: .75 >= .6 stops at 1 slot
+        0.5: ([1, 0, -1, -1], [1.5, 1.0, 0, 0]),                      # thr 1.0: 1.25 stops at 2
+        0.7: ([1, 0, 3, -1], [2.5 * .75 / 1.75, 2.5 * .5 / 1.75, 2.5 * .5 / 1.75, 0]),  # thr 1.4
+        0.9: ([1, 0, 3, 2], [2.5 * .75 / 2, 2.5 * .5 / 2, 2.5 * .5 / 2, 2.5 * .25 / 2]),  # thr 1.8: all
+        0.0: ([1, 0, 3, 2], [0.9375, 0.625, 0.625, 0.3125]),          # off
+        1.0: ([1, 0, 3, 2], [0.9375, 0.625, 0.625, 0.3125]),          # off
+    }
+    for p, (want_idx, want_w) in cases.items():
+        idx, w = O.route(x[:1], wr, bias, k=4, routed_scale=2.5, topp=p)
+        np.testing.assert_array_equal(idx[0], want_idx, err_msg=str(p))
+        np.testing.assert_allclose(w[0], want_w, rtol=1e-6, atol=0, err_msg=str(p))
+    # token 1 (all scores exactly 1/2): at p = .5 the first two slots sum to
+    # exactly p: the prefix that reaches p is kept, the next slot dropped
+    idx, w = O.route(x[1:2], wr, bias, k=4, routed_scale=2.5, topp=0.5)
+    np.testing.assert_array_equal(idx[0], [0, 1, -1, -1])
+    np.testing.assert_allclose(w[0], [1.25, 1.25, 0, 0])
+
+
+@pytest.mark.parametrize("E,k,d,T", [(16, 5, 24, 9), (33, 8, 40, 6)])
+def test_topp_invariants(E, k, d, T):
+    rng = np.random.default_rng(7 * E + k)
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    wr = (0.5 * rng.standard_normal((E, d))).astype(np.float32)
+    bias = (0.05 * rng.standard_normal(E)).astype(np.float32)
+    full, wfull, _, s, _ = O.route(x, wr, bias, k, 2.5, want_scores=True)
+    prev = np.ones(T, int)
+    for p in (1e-6, 0.2, 0.4, 0.6, 0.8, 0.95):
+        idx, w = O.route(x, wr, bias, k, 2.5, topp=p)
+        for t in range(T):
+            m = int((idx[t] >= 0).sum())
+            assert m >= 1 and (idx[t][:m] >= 0).all() and (idx[t][m:] == -1).all()  # a kept prefix
+            np.testing.assert_array_equal(idx[t][:m], full[t][:m])  # the selection order is untouched
+            assert m >= prev[t]  # more slots as p grows
+            prev[t] = m
+            st = s[t, full[t]].astype(np.float64)
+            q = np.cumsum(st) / st.sum()
+            assert q[m - 1] >= p - 1e-6 and (m == 1 or q[m - 2] < p + 1e-6)  # the smallest prefix reaching p
+            np.testing.assert_allclose(w[t][:m].sum(), 2.5, rtol=1e-12)
+            np.testing.assert_allclose(w[t][:m], 2.5 * st[:m] / st[:m].sum(), rtol=1e-12)
+            assert (w[t][m:] == 0).all()
+        if p == 1e-6:
+            assert (prev == 1).all()
+
+
+def test_topp_layer_drops_the_truncated_experts():
+    """The layer with truncation equals the weighted sum over the kept slots
+    of the single-expert outputs (plus the shared expert)."""
+    rng = np.random.default_rng(11)
+    d, f, E, k, T, wb = 32, 16, 6, 4, 3, 4
+    blobs = [rng.integers(0, 256, 3 * d * f * wb // 8, dtype=np.uint8) for _ in range(E + 1)]
+    scales = [np.exp(-4 + 0.3 * rng.standard_normal(2 * f + d)).astype(np.float32) for _ in range(E + 1)]
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    wr = (0.5 * rng.standard_normal((E, d))).astype(np.float32)
+    bias = np.zeros(E, np.float32)
+    r = O.layer(d, f, E, k, 1, wb, 2.5, blobs, scales, wr, bias, x, topp=0.55)
+    idx, w = O.route(x, wr, bias, k, 2.5, topp=0.55)
+    np.testing.assert_array_equal(r["idx"], idx)
+    assert (idx == -1).any() and (idx >= 0).any()
+    xq, sx = O.quantize(x)
+    for t in range(T):
+        want = O.expert(d, f, wb, blobs[E], scales[E], xq[t:t + 1], sx[t:t + 1])["y"][0].copy()
+        for j in range(k):
+            if idx[t, j] >= 0:
+                want += w[t, j] * O.expert(d, f, wb, blobs[idx[t, j]], scales[idx[t, j]], xq[t:t + 1],
+                                           sx[t:t + 1])["y"][0]
+        np.testing.assert_allclose(r["out"][t], want, rtol=1e-12, atol=1e-12)

@@ -142,6 +142,7 @@ class Workload:
     routed_scale: float = 2.5
     bias_halfwidth: float = 0.01
     residual: bool = False
+    topp: float = 0.0     # TOPK/TOPP truncation threshold of the router (0 = off)
 
     @property
     def blob_bytes(self) -> int:
