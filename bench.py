@@ -53,6 +53,9 @@ def parse(argv=None):
     ap.add_argument("--n-experts", type=int, default=0,
                     help="profiling case: the same layer with fewer routed experts (smaller pool)")
     ap.add_argument("--layers", type=int, default=0, help="profiling case: the first N layers of a stack")
+    ap.add_argument("--topp", type=float, default=0.0,
+                    help="supplementary case: the router's TOPK/TOPP truncation at this threshold "
+                         "(moe_config.topp; fewer experts per token)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="supplementary case: the workload with this many tokens per step (e.g. prefill at 8192)")
     ap.add_argument("--path", choices=["auto", "multi", "decode", "tc"], default="auto",
@@ -199,7 +202,7 @@ class OracleRunner:
 
     def _blobs(self, l, idx):
         wl, W = self.wl, self.W
-        need = set(idx.reshape(-1).tolist()) | ({wl.n_experts} if wl.has_shared else set())
+        need = (set(idx.reshape(-1).tolist()) - {-1}) | ({wl.n_experts} if wl.has_shared else set())
         blobs, scales = [None] * wl.n_blobs, [None] * wl.n_blobs
         sc = self.layers[l].scales.numpy()
         if len(self.cache) * wl.blob_bytes > self.cache_bytes:
@@ -220,11 +223,11 @@ class OracleRunner:
         for l in range(self.n_layers):
             L = self.layers[l]
             x_in = O.rmsnorm(xr) if stack else np.asarray(x, np.float32)
-            idx, _ = O.route(x_in, L.w_router, L.bias, wl.top_k, wl.routed_scale)
+            idx, _ = O.route(x_in, L.w_router, L.bias, wl.top_k, wl.routed_scale, topp=wl.topp)
             blobs, scales = self._blobs(l, idx)  # generation: not timed
             t0 = time.perf_counter()
             r = O.layer(wl.d, wl.f, wl.n_experts, wl.top_k, wl.has_shared, wl.wbits, wl.routed_scale, blobs, scales,
-                        L.w_router, L.bias, x_in)
+                        L.w_router, L.bias, x_in, topp=wl.topp)
             spent += time.perf_counter() - t0
             xr = xr + r["out"] if stack else r["out"]
         return spent
@@ -379,7 +382,8 @@ def gpu_arm(args, wl):
     T = wl.T
     n_layers = args.layers or wl.n_layers
     stack = n_layers > 1 or wl.residual
-    cfg = M.config(wl.d, wl.f, wl.n_experts, wl.top_k, wl.has_shared, wl.wbits, wl.routed_scale)
+    cfg = M.config(wl.d, wl.f, wl.n_experts, wl.top_k, wl.has_shared, wl.wbits, wl.routed_scale,
+                   topp=wl.topp)
     layers = [W.device_layer(wl, 0, l, dev) for l in range(n_layers)]
     pools = [M.make_pool(dl.pool_w, dl.pool_s) for dl in layers]
     n_sets = wl.n_token_sets if wl.n_token_sets > 1 else 4
@@ -487,7 +491,8 @@ def gpu_arm(args, wl):
 
     # unique experts per layer call (dedupe: each selected expert is read once)
     il = idx_log.cpu().numpy()
-    uniq = [len(set(il[i][l].reshape(-1).tolist())) + wl.has_shared for i in range(K) for l in range(n_layers)]
+    uniq = [len(set(il[i][l].reshape(-1).tolist()) - {-1}) + wl.has_shared  # -1: a slot TOPP dropped
+            for i in range(K) for l in range(n_layers)]
     gu_b, dn_b = expert_bytes(wl)
     step_exp_bytes = sum(u * (gu_b + dn_b) for u in uniq) / K  # counted expert bytes per step
     max_ms = max_over_ranks(total_ms, world, dist, dev)
@@ -719,6 +724,8 @@ def main(argv=None):
         wl = wl.replace(n_experts=args.n_experts, name=f"{wl.name}_e{args.n_experts}")
     if args.tokens:
         wl = wl.replace(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
+    if args.topp:
+        wl = wl.replace(topp=args.topp, name=f"{wl.name}_topp{args.topp:g}")
     if args.impl == "reference":
         reference_arm(args, wl)
     else:

@@ -37,7 +37,7 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("n_experts", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("has_shared", ctypes.c_int32), ("wbits", ctypes.c_int32),
-                ("routed_scale", ctypes.c_float), ("tc_min_tokens", ctypes.c_int32)]
+                ("routed_scale", ctypes.c_float), ("tc_min_tokens", ctypes.c_int32), ("topp", ctypes.c_float)]
 
     @property
     def blob_bytes(self) -> int:
@@ -63,8 +63,8 @@ class MoePool(ctypes.Structure):
 
 
 def config(d: int, f: int, n_experts: int, top_k: int, has_shared: int = 1, wbits: int = 4,
-           routed_scale: float = 2.5, tc_min_tokens: int = 0) -> MoeConfig:
-    return MoeConfig(d, f, n_experts, top_k, has_shared, wbits, routed_scale, tc_min_tokens)
+           routed_scale: float = 2.5, tc_min_tokens: int = 0, topp: float = 0.0) -> MoeConfig:
+    return MoeConfig(d, f, n_experts, top_k, has_shared, wbits, routed_scale, tc_min_tokens, topp)
 
 
 def _load() -> ctypes.CDLL:

@@ -120,6 +120,7 @@ moe_status check_cfg(const moe_config* c) {
         return fail(MOE_EINVAL, "top_k must be in [1, min(n_experts, 32)]");
     if (c->has_shared != 0 && c->has_shared != 1) return fail(MOE_EINVAL, "has_shared must be 0 or 1");
     if (!(c->routed_scale == c->routed_scale)) return fail(MOE_EINVAL, "routed_scale is NaN");
+    if (!(c->topp >= 0.0f && c->topp <= 1.0f)) return fail(MOE_EINVAL, "topp must be in [0, 1]");
     return MOE_OK;
 }
 
@@ -166,6 +167,7 @@ static Params base_params(const moe_config* c, const Dims& m, void* ws, size_t w
     p.wait_ns = kWaitLimitNs;
     p.skip_h_task = -1;
     p.routed_scale = c->routed_scale;
+    p.topp = c->topp;
     p.blob_bytes = 3ll * c->d * c->f * c->wbits / 8;
     p.scale_rows = 2 * c->f + c->d;
     p.CH = pick_ch(m.T);

@@ -168,6 +168,7 @@ struct Params {
     unsigned long long* trace;  // optional per-CTA phase stamps of the decode kernel
     unsigned long long wait_ns; // bound of the decode kernel's device-side waits (its slot waits: twice this)
     int skip_h_task;            // testing: the one-token decode leaves this task's h unwritten (-1 = none)
+    float topp;                 // TOPK/TOPP truncation of the router (0 or 1 = off)
     const float* w_router;
     const float* bias;
     float* out;
@@ -269,6 +270,24 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                      smem_u32(dst)),
                  "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
+}
+// TOPK/TOPP truncation of one warp's k selected slots (lane j holds slot j).
+// With 0 < topp < 1, slot j is kept iff j == 0 or cex -- the float sum of the
+// scores of slots 0..j-1, added in slot order -- is below fl(topp * ssum),
+// ssum the float sum over all k slots: the smallest prefix whose normalised
+// scores reach topp.  Returns the normaliser of the kept weights, cin (the
+// inclusive sum) of the last kept slot.  Any other topp keeps every slot and
+// returns ssum.  topp is the same for the whole warp.
+__device__ __forceinline__ float topp_keep(float topp, int k, float ssum, float cex, float cin, bool& kept) {
+    const int lane = threadIdx.x & 31;
+    if (!(topp > 0.0f && topp < 1.0f)) {
+        kept = lane < k;
+        return ssum;
+    }
+    const float thr = __fmul_rn(topp, ssum);
+    kept = lane < k && (lane == 0 || cex < thr);
+    const int m = __popc(__ballot_sync(0xffffffffu, kept));
+    return __shfl_sync(0xffffffffu, cin, m - 1);
 }
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;

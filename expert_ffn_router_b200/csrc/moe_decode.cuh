@@ -194,10 +194,10 @@ __device__ __forceinline__ uint2 route_pair(float logit, float bias) {
 }
 
 // Top-k of one token by one warp from its row of (selection, score) pairs in
-// global memory; lane j (< k) returns slot j's expert and weight.  Same rule
-// as topk_token.
-__device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float scale, float* s_sm, float* sel_sm,
-                                          int& my_e, float& my_w) {
+// global memory; lane j (< k) returns slot j's expert and weight (-1 and 0 for
+// a slot the TOPP truncation drops).  Same rule as topk_token.
+__device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float scale, float topp, float* s_sm,
+                                          float* sel_sm, int& my_e, float& my_w) {
     const int lane = threadIdx.x & 31;
     for (int e = lane; e < E; e += 32) {
         const uint2 pr = __ldcg(prow + e);
@@ -205,7 +205,7 @@ __device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float
         sel_sm[e] = __uint_as_float(pr.x);
     }
     __syncwarp();
-    float ssum = 0.0f, my_s = 0.0f;
+    float ssum = 0.0f, my_s = 0.0f, cex = 0.0f, cin = 0.0f;
     my_e = 0;
     for (int j = 0; j < k; ++j) {
         float bv = -FLT_MAX;
@@ -230,13 +230,18 @@ __device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float
         if (lane == j) {
             my_e = be;
             my_s = sj;
+            cex = ssum;
         }
         ssum = __fadd_rn(ssum, sj);
+        if (lane == j) cin = ssum;
         __syncwarp();
         if (lane == 0) sel_sm[be] = -INFINITY;
         __syncwarp();
     }
-    my_w = lane < k ? __fmul_rn(__fdiv_rn(my_s, ssum), scale) : 0.0f;
+    bool kept;
+    const float norm = topp_keep(topp, k, ssum, cex, cin, kept);
+    my_w = kept ? __fmul_rn(__fdiv_rn(my_s, norm), scale) : 0.0f;
+    if (!kept) my_e = -1;
 }
 
 // NG / ND: 16-byte weight chunks per lane of a gate/up row / a down row when
@@ -246,7 +251,7 @@ __device__ __forceinline__ void topk_warp(const uint2* prow, int E, int k, float
 // Top-k of one token by one warp for E <= 256: lane l holds experts l + 32 i
 // in registers; each round takes the largest selection score (lowest index on
 // ties) with two warp reductions.  Same rule and arithmetic as topk_warp.
-__device__ __forceinline__ void topk_warp_small(const uint2* prow, int E, int k, float scale, int& my_e,
+__device__ __forceinline__ void topk_warp_small(const uint2* prow, int E, int k, float scale, float topp, int& my_e,
                                                 float& my_w, unsigned long long* tr) {
     const int lane = threadIdx.x & 31;
     float sv[8];
@@ -260,7 +265,7 @@ __device__ __forceinline__ void topk_warp_small(const uint2* prow, int E, int k,
         key[i] = lane + 32 * i < E ? float_key(__uint_as_float(pr[i].x)) : 0u;  // 0: below every real key
     }
     if (tr && lane == 0 && key[0] != 1u) *tr = global_timer_ns();  // once loaded (the branch reads a value)
-    float ssum = 0.0f, my_s = 0.0f;
+    float ssum = 0.0f, my_s = 0.0f, cex = 0.0f, cin = 0.0f;
     my_e = 0;
     for (int j = 0; j < k; ++j) {
         unsigned best = 0u;
@@ -287,10 +292,15 @@ __device__ __forceinline__ void topk_warp_small(const uint2* prow, int E, int k,
         if (lane == j) {
             my_e = e_win;
             my_s = sj;
+            cex = ssum;
         }
         ssum = __fadd_rn(ssum, sj);
+        if (lane == j) cin = ssum;
     }
-    my_w = lane < k ? __fmul_rn(__fdiv_rn(my_s, ssum), scale) : 0.0f;
+    bool kept;
+    const float norm = topp_keep(topp, k, ssum, cex, cin, kept);
+    my_w = kept ? __fmul_rn(__fdiv_rn(my_s, norm), scale) : 0.0f;
+    if (!kept) my_e = -1;
 }
 
 template <int WB, int TM, int NG, int ND, typename XT>
@@ -844,14 +854,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 float my_w;
                 if (E <= kDecBiasCache) {
                     topk_warp_small(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale,
-                                    my_e, my_w, trace && warp == 0 ? trace + 18 : nullptr);
+                                    p.topp, my_e, my_w, trace && warp == 0 ? trace + 18 : nullptr);
                 } else {
                     float* scr = reinterpret_cast<float*>(hsb) + (size_t)warp * 2 * E;
-                    topk_warp(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale, scr,
-                              scr + E, my_e, my_w);
+                    topk_warp(reinterpret_cast<const uint2*>(p.ws.logits) + (size_t)warp * E, E, k, p.routed_scale,
+                              p.topp, scr, scr + E, my_e, my_w);
                 }
                 if (lane < k) {
-                    my_e = idx_in(hdr, my_e, 0, E, 618);
+                    if (my_e != -1) my_e = idx_in(hdr, my_e, 0, E, 618);  // -1: dropped by the truncation
                     C.idx[warp][lane] = my_e;
                     C.w[warp][lane] = my_w;
                     if (c == 0) {
@@ -867,29 +877,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             // bucket: sort the T*k assignments by (expert, token, slot); one task per expert
             const int A = T * k;
             if (T == 1) {  // one token: the k experts, each a task with that token, by ascending expert
-                if (warp == 0) {
-                    const int e = lane < k ? C.idx[0][lane] : 0x7fffffff;
+                if (warp == 0) {  // (a slot the truncation dropped sorts last and makes no task)
+                    const int e = lane < k && C.idx[0][lane] >= 0 ? C.idx[0][lane] : 0x7fffffff;
                     int rank = 0;
                     for (int jj = 0; jj < k; ++jj) rank += __shfl_sync(kFull, e, jj) < e;
-                    if (lane < k) {
+                    const bool kept = e != 0x7fffffff;
+                    if (kept) {
                         C.ttok[HS + rank][0] = lane;  // assignment id: token 0, slot lane
                         C.tasks[HS + rank] = make_int4(e, 1, 0, 0);
                     }
-                    if (lane == 0) C.n_tasks = HS + k;
+                    const int m = __popc(__ballot_sync(kFull, kept));
+                    if (lane == 0) C.n_tasks = HS + m;
                 }
             } else if (ctid < A) {
-                const int ea = C.idx[ctid / k][ctid % k];
+                // a slot the truncation dropped (-1) sorts last, as expert E
+                const int ea = C.idx[ctid / k][ctid % k] < 0 ? E : C.idx[ctid / k][ctid % k];
                 int pos = 0, a2 = 0;
                 for (int t2 = 0; t2 < T; ++t2)
                     for (int j2 = 0; j2 < k; ++j2, ++a2) {
-                        const int e2 = C.idx[t2][j2];
+                        const int e2 = C.idx[t2][j2] < 0 ? E : C.idx[t2][j2];
                         pos += (e2 < ea) || (e2 == ea && a2 < ctid);
                     }
                 C.sorted[pos] = ctid;
                 C.sorted_e[pos] = ea;
             }
             named_sync(kDecBar, kDecCons);
-            if (T > 1 && ctid < A) {
+            if (T > 1 && ctid < A && C.sorted_e[ctid] < E) {
                 const int a = C.sorted[ctid];
                 const int ea = C.sorted_e[ctid];
                 int tq = -1, rank = 0, n = 0;
@@ -901,7 +914,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 for (int q = 0; q < A; ++q) n += C.sorted_e[q] == ea;
                 C.ttok[HS + tq][rank] = (a / k) * S + (a % k);
                 if (rank == 0) C.tasks[HS + tq] = make_int4(ea, n, 0, 0);
-                if (ctid == A - 1) C.n_tasks = HS + tq + 1;
+                if (ctid == A - 1 || C.sorted_e[ctid + 1] == E) C.n_tasks = HS + tq + 1;  // the last kept one
             }
             named_sync(kDecBar, kDecCons);
             if (ctid == 0) {
@@ -1107,7 +1120,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             if (ctid == 0) DEC_TRACE(21);
             for (int rl = ctid; rl < rr_rows; rl += kDecCons) {
                 float o = 0.0f;
-                for (int jj = 0; jj < k; ++jj) o = fmaf(C.w[0][jj], ys[jj * RRW + rl], o);
+                for (int jj = 0; jj < k; ++jj)
+                    if (C.idx[0][jj] >= 0) o = fmaf(C.w[0][jj], ys[jj * RRW + rl], o);
                 if (HS) o += ys[k * RRW + rl];
                 float* dst = p.out + rr_lo + rl;
                 *dst = p.accumulate ? *dst + o : o;
@@ -1277,7 +1291,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 const int t = i / rows, r = r0 + i % rows;
                 float o = 0.0f;
                 for (int jj = 0; jj < k; ++jj)
-                    o = fmaf(C.w[t][jj], __ldcg(p.ws.ybuf + ((size_t)t * S + jj) * d + r), o);
+                    if (C.idx[t][jj] >= 0) o = fmaf(C.w[t][jj], __ldcg(p.ws.ybuf + ((size_t)t * S + jj) * d + r), o);
                 if (HS) o += __ldcg(p.ws.ybuf + ((size_t)t * S + k) * d + r);
                 float* dst = p.out + (size_t)t * d + r;
                 *dst = p.accumulate ? *dst + o : o;

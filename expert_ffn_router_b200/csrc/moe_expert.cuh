@@ -274,8 +274,9 @@ __global__ void __launch_bounds__(kThreads) k_down(const Params p) {
             for (int i = tid; i < T * rows; i += kThreads) {
                 const int t = i / rows, r = rb * RB + i % rows;
                 float o = 0.0f;
-                for (int j = 0; j < k; ++j)
-                    o = fmaf(__ldcg(p.ws.w + (size_t)t * k + j), __ldcg(p.ws.ybuf + ((size_t)t * S + j) * d + r), o);
+                for (int j = 0; j < k; ++j)  // (a slot the truncation dropped has no output)
+                    if (__ldcg(p.ws.idx + (size_t)t * k + j) >= 0)
+                        o = fmaf(__ldcg(p.ws.w + (size_t)t * k + j), __ldcg(p.ws.ybuf + ((size_t)t * S + j) * d + r), o);
                 if (p.m.has_shared) o += __ldcg(p.ws.ybuf + ((size_t)t * S + k) * d + r);
                 float* dst = p.out + (size_t)t * d + r;
                 *dst = p.accumulate ? *dst + o : o;

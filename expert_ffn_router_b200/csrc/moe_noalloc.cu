@@ -76,6 +76,7 @@ extern "C" moe_status moe_route_static(const moe_config* cfg, const void* x, moe
     p.m = Dims{cfg->d, cfg->f, cfg->n_experts, cfg->top_k, cfg->has_shared, cfg->wbits, T,
                cfg->top_k + cfg->has_shared};
     p.routed_scale = cfg->routed_scale;
+    p.topp = cfg->topp;
     p.ksplit = 1;
     char* b = static_cast<char*>(base);
     p.ws.hdr = reinterpret_cast<WsHeader*>(b);

@@ -94,7 +94,7 @@ static __device__ void topk_token(const Params& p, int t, float* s_sm, float* se
         sel_sm[e] = __fadd_rn(s, __ldg(p.bias + e));
     }
     __syncwarp();
-    float ssum = 0.0f, my_s = 0.0f;
+    float ssum = 0.0f, my_s = 0.0f, cex = 0.0f, cin = 0.0f;
     int my_e = 0;
     for (int j = 0; j < k; ++j) {
         float bv = -FLT_MAX;
@@ -119,17 +119,22 @@ static __device__ void topk_token(const Params& p, int t, float* s_sm, float* se
         if (lane == j) {
             my_e = be;
             my_s = sj;
+            cex = ssum;
         }
         ssum = __fadd_rn(ssum, sj);
+        if (lane == j) cin = ssum;
         __syncwarp();
         if (lane == 0) sel_sm[be] = -INFINITY;
         __syncwarp();
     }
-    if (lane < k) {
-        const float w = __fmul_rn(__fdiv_rn(my_s, ssum), p.routed_scale);
-        p.ws.idx[(size_t)t * k + lane] = my_e;
+    bool kept;
+    const float norm = topp_keep(p.topp, k, ssum, cex, cin, kept);
+    if (lane < k) {  // a slot the truncation drops selects no expert: -1, weight 0
+        const float w = kept ? __fmul_rn(__fdiv_rn(my_s, norm), p.routed_scale) : 0.0f;
+        const int e = kept ? my_e : -1;
+        p.ws.idx[(size_t)t * k + lane] = e;
         p.ws.w[(size_t)t * k + lane] = w;
-        if (p.idx_out) p.idx_out[(size_t)t * k + lane] = my_e;
+        if (p.idx_out) p.idx_out[(size_t)t * k + lane] = e;
         if (p.w_out) p.w_out[(size_t)t * k + lane] = w;
     }
 }
@@ -173,7 +178,9 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
             for (int u = 0; u < 4; ++u) {
                 const int i = i0 + tid + u * kThreads;
                 if (i < nb) {
-                    if (v[u] < 0 || v[u] >= E) {
+                    if (v[u] == -1) {
+                        v[u] = E;  // a slot the truncation dropped: no assignment
+                    } else if (v[u] < 0 || v[u] >= E) {
                         set_status(hdr, MOE_EDEVICE, base + i);
                         v[u] = 0;
                     }
@@ -188,7 +195,8 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
         const int nb = min(kBucketStage, A - base);
         load_stage(base, nb);
         __syncthreads();
-        for (int i = tid; i < nb; i += kThreads) atomicAdd(&cnt[stage[i]], 1);
+        for (int i = tid; i < nb; i += kThreads)
+            if (stage[i] < E) atomicAdd(&cnt[stage[i]], 1);
         __syncthreads();
     }
     for (int e = tid; e < E; e += kThreads) {
@@ -218,7 +226,7 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
         for (int b = lo; b < hi; b += 32) {  // per-warp histogram of the slice
             const int e = b + lane < hi ? stage[b + lane] : E;
             const unsigned peers = __match_any_sync(kFull, e);
-            if (b + lane < hi && (peers & lanemask_lt()) == 0) hist[warp * E + e] += __popc(peers);
+            if (e < E && (peers & lanemask_lt()) == 0) hist[warp * E + e] += __popc(peers);
             __syncwarp();
         }
         __syncthreads();
@@ -238,9 +246,9 @@ static __device__ void bucket_cta(const Params& p, int* smem) {
             const int e = b + lane < hi ? stage[b + lane] : E;
             const unsigned peers = __match_any_sync(kFull, e);
             const int rank = __popc(peers & lanemask_lt());
-            if (b + lane < hi) p.ws.asg[asg_base + hist[warp * E + e] + rank] = (a / k) * S + (a % k);
+            if (e < E) p.ws.asg[asg_base + hist[warp * E + e] + rank] = (a / k) * S + (a % k);
             __syncwarp();
-            if (b + lane < hi && rank == 0) hist[warp * E + e] += __popc(peers);
+            if (e < E && rank == 0) hist[warp * E + e] += __popc(peers);
             __syncwarp();
         }
         __syncthreads();
@@ -480,7 +488,7 @@ __global__ void __launch_bounds__(kThreads) k_topk_small(const Params p, int buc
                 key[i] = float_key(__fadd_rn(sv[i], __ldg(p.bias + e)));
             }
         }
-        float ssum = 0.0f, my_s = 0.0f;
+        float ssum = 0.0f, my_s = 0.0f, cex = 0.0f, cin = 0.0f;
         int my_e = 0;
         for (int j = 0; j < k; ++j) {
             unsigned best = 0u;
@@ -507,14 +515,19 @@ __global__ void __launch_bounds__(kThreads) k_topk_small(const Params p, int buc
             if (lane == j) {
                 my_e = e_win;
                 my_s = sj;
+                cex = ssum;
             }
             ssum = __fadd_rn(ssum, sj);
+            if (lane == j) cin = ssum;
         }
-        if (lane < k) {
-            const float w = __fmul_rn(__fdiv_rn(my_s, ssum), p.routed_scale);
-            p.ws.idx[(size_t)t * k + lane] = my_e;
+        bool kept;
+        const float norm = topp_keep(p.topp, k, ssum, cex, cin, kept);
+        if (lane < k) {  // a slot the truncation drops selects no expert: -1, weight 0
+            const float w = kept ? __fmul_rn(__fdiv_rn(my_s, norm), p.routed_scale) : 0.0f;
+            const int e = kept ? my_e : -1;
+            p.ws.idx[(size_t)t * k + lane] = e;
             p.ws.w[(size_t)t * k + lane] = w;
-            if (p.idx_out) p.idx_out[(size_t)t * k + lane] = my_e;
+            if (p.idx_out) p.idx_out[(size_t)t * k + lane] = e;
             if (p.w_out) p.w_out[(size_t)t * k + lane] = w;
         }
     }

@@ -531,6 +531,7 @@ __global__ void __launch_bounds__(kThreads) k_combine(const Params p) {
         const int t = (int)(i / nq), c4 = (int)(i - (size_t)t * nq) * 4;
         float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         for (int j = 0; j < k; ++j) {
+            if (__ldcg(p.ws.idx + (size_t)t * k + j) < 0) continue;  // dropped by the truncation: no output
             const float w = __ldcg(p.ws.w + (size_t)t * k + j);
             const float4 y = __ldcg(reinterpret_cast<const float4*>(p.ws.ybuf + ((size_t)t * S + j) * d + c4));
             o.x = fmaf(w, y.x, o.x);

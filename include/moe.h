@@ -79,12 +79,24 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  *  moe_expert_ffn, moe_expert_down); 0 = library default (3: on B200 at the
  *  GLM-5.2 expert shape the single-launch decode kernel is faster for one and
  *  two tokens, the tensor-core path from three on), < 0 = never.
+ *  topp: TOPK/TOPP truncation of the router, opt-in (0 or 1 = off, the
+ *  router as above).  With 0 < topp < 1 each token keeps the smallest prefix
+ *  of its k selected slots (selection order) whose scores, normalised over
+ *  the k, sum to at least topp: slot j is kept iff j == 0 or the float32 sum
+ *  of the scores of slots 0..j-1, added in slot order, is below
+ *  float32(topp * sum of all k).  A dropped slot selects no expert: its
+ *  topk_idx is -1, its weight 0, and no expert is read for it; the kept
+ *  weights are the kept scores over their sum, times routed_scale.  (A
+ *  reading of the pages' TOPP option: agentlenshq, benchmark table, the
+ *  --topp 0.7 rows; takumi3488, the TOPK / TOPP options of the run logs.)
  * Limits (MOE_EINVAL otherwise): 1 <= k <= min(E, 32); E <= 1024;
- * d * wbits / 8 and f * wbits / 8 multiples of 16; d <= 8192; f <= 8192. */
+ * d * wbits / 8 and f * wbits / 8 multiples of 16; d <= 8192; f <= 8192;
+ * 0 <= topp <= 1. */
 typedef struct {
     int32_t d, f, n_experts, top_k, has_shared, wbits;
     float routed_scale;
     int32_t tc_min_tokens;
+    float topp;
 } moe_config;
 
 /* One layer's experts, resident in device memory, canonical layout.

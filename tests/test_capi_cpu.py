@@ -38,7 +38,8 @@ def test_workspace_bytes():
 
 
 @pytest.mark.parametrize("field,value", [("wbits", 3), ("d", 100), ("f", 40), ("top_k", 0), ("top_k", 9),
-                                         ("n_experts", 0), ("has_shared", 2), ("d", 16384)])
+                                         ("n_experts", 0), ("has_shared", 2), ("d", 16384), ("topp", -0.1),
+                                         ("topp", 1.5), ("topp", float("nan"))])
 def test_layer_rejects_bad_config(field, value):
     c = good_cfg(**{field: value})
     pool = M.MoePool(FAKE, FAKE)
