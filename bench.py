@@ -53,6 +53,9 @@ def parse(argv=None):
     ap.add_argument("--n-experts", type=int, default=0,
                     help="profiling case: the same layer with fewer routed experts (smaller pool)")
     ap.add_argument("--layers", type=int, default=0, help="profiling case: the first N layers of a stack")
+    ap.add_argument("--cache-slots", type=int, default=0,
+                    help="supplementary case: the layer's pool in pinned host memory behind an HBM expert cache "
+                         "of this many slots (moe_cache_fetch); reports hit rate and host->device bytes per token")
     ap.add_argument("--topp", type=float, default=0.0,
                     help="supplementary case: the router's TOPK/TOPP truncation at this threshold "
                          "(moe_config.topp; fewer experts per token)")
@@ -670,6 +673,67 @@ def e2e_arm(args, wl, M, torch, dist, world, dev, stream, toks, xbuf, out, run_s
                                  "stream synchronised every step (L2 flushed before each step, not timed)"}}
 
 
+def cache_arm(args, wl):
+    """One layer, T tokens per call, with its pool in pinned host memory behind
+    an HBM expert cache: each step routes, copies the indices to the host,
+    fetches the missing experts (one DMA copy each) and runs the layer on the
+    cached pool; timed by the host clock per synchronised step (the fetch
+    needs the routing on the host).  Reports tokens/s, the hit rate and the
+    host -> device bytes per token."""
+    import torch
+    import expert_ffn_router_b200 as M
+    import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    K, Wm, T = args.steps, args.warmup, wl.T
+    cfg = M.config(wl.d, wl.f, wl.n_experts, wl.top_k, wl.has_shared, wl.wbits, wl.routed_scale, topp=wl.topp)
+    dl = W.device_layer(wl, 0, 0, dev)
+    host_w = dl.pool_w.cpu().pin_memory()
+    del dl.pool_w  # only the cache's slots stay in HBM
+    torch.cuda.empty_cache()
+    cache = M.ExpertCache(cfg, host_w, dl.pool_s, args.cache_slots, dev)
+    n_sets = wl.n_token_sets if wl.n_token_sets > 1 else 4
+    toks = torch.stack([W.tokens(wl, 0, s) for s in range(n_sets)]).to(dev)
+    ws = M.workspace(cfg, T, dev)
+    out = torch.empty(T, wl.d, device=dev)
+    idx = torch.empty(T, wl.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, wl.top_k, device=dev)
+    idx_h = torch.empty(T, wl.top_k, dtype=torch.int32).pin_memory()
+
+    def step(i):
+        x = toks[i % n_sets]
+        M.moe_route(cfg, x, dl.w_router, dl.bias, idx, w, ws)
+        idx_h.copy_(idx, non_blocking=True)
+        torch.cuda.synchronize()
+        st = cache.fetch(idx_h)
+        M.moe_layer(cfg, cache.pool, dl.w_router, dl.bias, x, out, ws)
+        torch.cuda.synchronize()
+        return st
+
+    for i in range(Wm):
+        step(i)
+    wall, hits, misses, nbytes = [], 0, 0, 0
+    for i in range(K):
+        t0 = time.perf_counter()
+        st = step(Wm + i)
+        wall.append(time.perf_counter() - t0)
+        hits, misses, nbytes = hits + st.hits, misses + st.misses, nbytes + st.bytes
+    assert M.moe_poll_status(ws) == M.MOE_OK
+    total = sum(wall)
+    line = {"metric": "MoE-layer decode tokens/s with an HBM expert cache (pool in pinned host memory)",
+            "value": K * T / total, "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": Wm,
+            "ms_per_step": 1e3 * total / K, "step_ms_median": 1e3 * statistics.median(wall),
+            "higher_is_better": True, "dtype": "i8*i4->i32" if wl.wbits == 4 else "i8*i2->i32",
+            "data": "synthetic", "config": {"workload": wl.name, "T": T, "experts": wl.n_experts,
+                                            "top_k": wl.top_k, "cache_slots": args.cache_slots,
+                                            "pool_gb": (wl.n_experts + wl.has_shared) * cfg.blob_bytes / 1e9},
+            "cache": {"hit_rate": hits / max(1, hits + misses), "hits": hits, "misses": misses,
+                      "h2d_bytes_per_token": nbytes / (K * T), "h2d_gbs": nbytes / total / 1e9},
+            "how": "host clock per step: route, indices to the host, moe_cache_fetch (one DMA copy per missing "
+                   "expert), moe_layer on the cached pool, synchronised; no L2 flush (the copies dominate)"}
+    print(json.dumps(line), flush=True)
+
+
 def int8_peak(path):
     """Dense int8 x int8 -> int32 GEMM throughput of the device (cuBLAS through
     torch._int_mm, 8192 x 8192 x 8192), CUDA events after warm-up: the
@@ -728,6 +792,8 @@ def main(argv=None):
         wl = wl.replace(topp=args.topp, name=f"{wl.name}_topp{args.topp:g}")
     if args.impl == "reference":
         reference_arm(args, wl)
+    elif args.cache_slots:
+        cache_arm(args, wl)
     else:
         gpu_arm(args, wl)
 

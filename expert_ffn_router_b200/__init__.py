@@ -59,7 +59,17 @@ class MoeLayerOpts(ctypes.Structure):
 
 
 class MoePool(ctypes.Structure):
-    _fields_ = [("w", ctypes.c_void_p), ("s", ctypes.c_void_p)]
+    _fields_ = [("w", ctypes.c_void_p), ("s", ctypes.c_void_p), ("slot_of", ctypes.c_void_p),
+                ("n_slots", ctypes.c_int32)]
+
+
+class MoeCache(ctypes.Structure):
+    _fields_ = [("host_w", ctypes.c_void_p), ("slots", ctypes.c_void_p), ("slot_of", ctypes.c_void_p),
+                ("state", ctypes.c_void_p), ("n_slots", ctypes.c_int32)]
+
+
+class MoeCacheStats(ctypes.Structure):
+    _fields_ = [("hits", ctypes.c_int64), ("misses", ctypes.c_int64), ("bytes", ctypes.c_int64)]
 
 
 def config(d: int, f: int, n_experts: int, top_k: int, has_shared: int = 1, wbits: int = 4,
@@ -86,6 +96,9 @@ def _load() -> ctypes.CDLL:
         "moe_layer_ex": (I32, [C, PL, P, P, P, I32, I32, P, I32, P, P, P, SZ, P, ctypes.POINTER(MoeLayerOpts)]),
         "moe_rmsnorm": (I32, [P, I32, I32, I32, F, P, P, P]),
         "moe_poll_status": (I32, [P, ctypes.POINTER(I32), P]),
+        "moe_cache_state_bytes": (SZ, [C, I32]),
+        "moe_cache_init": (I32, [C, ctypes.POINTER(MoeCache), P]),
+        "moe_cache_fetch": (I32, [C, ctypes.POINTER(MoeCache), P, I32, P, ctypes.POINTER(MoeCacheStats)]),
         "moe_status_string": (ctypes.c_char_p, [I32]),
         "moe_last_error": (ctypes.c_char_p, []),
     }
@@ -141,12 +154,52 @@ def _xdtype(x: torch.Tensor) -> int:
     raise ValueError(f"x must be float32 or bfloat16, got {x.dtype}")
 
 
-def make_pool(w: torch.Tensor, s: torch.Tensor) -> MoePool:
-    """The C struct over two device tensors; it keeps references to them, so
-    their memory stays allocated for as long as the struct is in use."""
-    pool = MoePool(_ptr(w, torch.uint8, name="pool.w"), _ptr(s, torch.float32, name="pool.s"))
-    pool._tensors = (w, s)
+def make_pool(w: torch.Tensor, s: torch.Tensor, slot_of: Optional[torch.Tensor] = None,
+              n_slots: int = 0) -> MoePool:
+    """The C struct over device tensors; it keeps references to them, so their
+    memory stays allocated for as long as the struct is in use.  With
+    ``slot_of`` (an HBM expert cache's slot table) ``w`` holds ``n_slots``
+    blobs."""
+    pool = MoePool(_ptr(w, torch.uint8, name="pool.w"), _ptr(s, torch.float32, name="pool.s"),
+                   _ptr(slot_of, torch.int32, name="pool.slot_of"), n_slots if slot_of is not None else 0)
+    pool._tensors = (w, s, slot_of)
     return pool
+
+
+class ExpertCache:
+    """An HBM expert cache over one layer's pool in pinned host memory
+    (moe_cache_init / moe_cache_fetch): ``n_slots`` device blobs, the slot
+    table and the host book-keeping, all owned here.  ``pool`` is the
+    moe_pool over the slots to pass to moe_layer after ``fetch``."""
+
+    def __init__(self, cfg: MoeConfig, host_w: torch.Tensor, scales: torch.Tensor, n_slots: int, device="cuda",
+                 stream=None):
+        if host_w.is_cuda or not host_w.is_pinned():
+            raise ValueError("host_w: expected a pinned host tensor")
+        self.cfg = cfg
+        B = cfg.blob_bytes
+        self.host_w = host_w
+        self.slots = torch.empty(n_slots * B, dtype=torch.uint8, device=device)
+        self.slot_of = torch.empty(cfg.n_experts + cfg.has_shared, dtype=torch.int32, device=device)
+        nb = lib.moe_cache_state_bytes(ctypes.byref(cfg), n_slots)
+        if nb == 0:
+            raise MoeError(MOE_EINVAL, "moe_cache_state_bytes", lib.moe_last_error().decode())
+        self.state = (ctypes.c_uint64 * ((nb + 7) // 8))()
+        self.c = MoeCache(host_w.data_ptr(), self.slots.data_ptr(), self.slot_of.data_ptr(),
+                          ctypes.addressof(self.state), n_slots)
+        self.pool = make_pool(self.slots, scales, self.slot_of, n_slots)
+        _check(lib.moe_cache_init(ctypes.byref(cfg), ctypes.byref(self.c), _stream(stream)), "moe_cache_init")
+
+    def fetch(self, idx_host: torch.Tensor, stream=None) -> MoeCacheStats:
+        """Makes the experts of ``idx_host`` (int32 [T][top_k] on the host)
+        resident; returns this call's hits, misses and copied bytes."""
+        idx_host = idx_host.contiguous()
+        if idx_host.is_cuda or idx_host.dtype != torch.int32:
+            raise ValueError("idx_host: expected an int32 host tensor")
+        st = MoeCacheStats()
+        _check(lib.moe_cache_fetch(ctypes.byref(self.cfg), ctypes.byref(self.c), idx_host.data_ptr(),
+                                   idx_host.shape[0], _stream(stream), ctypes.byref(st)), "moe_cache_fetch")
+        return st
 
 
 # ---------------------------------------------------------------------------

@@ -124,6 +124,14 @@ moe_status check_cfg(const moe_config* c) {
     return MOE_OK;
 }
 
+// A cached pool (slot_of set) holds n_slots >= 1 blobs; its table is device memory.
+static moe_status check_pool_slots(const moe_pool* pool) {
+    if (!pool->slot_of) return MOE_OK;
+    if (pool->n_slots < 1) return fail(MOE_EINVAL, "pool->n_slots must be >= 1 when pool->slot_of is set");
+    if (reinterpret_cast<uintptr_t>(pool->slot_of) % 4) return fail(MOE_EALIGN, "pool->slot_of is not 4-byte aligned");
+    return MOE_OK;
+}
+
 moe_status check_ptr(const void* p, const char* name, bool nullable) {
     if (!p) return nullable ? MOE_OK : fail(MOE_EINVAL, std::string(name) + " is NULL");
     if (!aligned16(p)) return fail(MOE_EALIGN, std::string(name) + " is not 16-byte aligned");
@@ -357,6 +365,7 @@ static moe_status expert_common(const moe_config* cfg, const moe_pool* pool, int
     MOE_TRY(check_cfg(cfg));
     if (!pool) return fail(MOE_EINVAL, "pool is NULL");
     MOE_TRY(check_ptr(pool->w, "pool->w"));
+    MOE_TRY(check_pool_slots(pool));
     MOE_TRY(check_ptr(pool->s, "pool->s"));
     if (T < 0) return fail(MOE_EINVAL, "T < 0");
     if (expert < -1 || expert >= cfg->n_experts) return fail(MOE_EINVAL, "expert out of range");
@@ -367,6 +376,8 @@ static moe_status expert_common(const moe_config* cfg, const moe_pool* pool, int
     Params p = base_params(cfg, m, ws, ws_bytes);
     p.pool = pool->w;
     p.scales = pool->s;
+    p.slot_of = pool->slot_of;
+    p.n_slots = pool->n_slots;
     p.direct_out = 1;
     p.out = y;
     *out_p = p;
@@ -391,6 +402,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const moe_pool* pool, int32_t e
     else if (dbg) p.CH = 8;
     p.pool = pool->w;
     p.scales = pool->s;
+    p.slot_of = pool->slot_of;
+    p.n_slots = pool->n_slots;
     p.direct_out = 1;
     p.out = y;
     p.dbg_acc_gu = dbg_acc_gu;
@@ -434,6 +447,8 @@ moe_status moe_expert_down(const moe_config* cfg, const moe_pool* pool, int32_t 
     else if (dbg) p.CH = 8;
     p.pool = pool->w;
     p.scales = pool->s;
+    p.slot_of = pool->slot_of;
+    p.n_slots = pool->n_slots;
     p.direct_out = 1;
     p.out = y;
     p.hq_in = hq;
@@ -496,6 +511,7 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     const int io = opts ? opts->io_host : 0;
     if (T == 0) return MOE_OK;
     MOE_TRY(check_ptr(pool->w, "pool->w"));
+    MOE_TRY(check_pool_slots(pool));
     MOE_TRY(check_ptr(pool->s, "pool->s"));
     MOE_TRY(check_ptr(w_router, "w_router"));
     MOE_TRY(check_ptr(bias, "bias"));
@@ -516,6 +532,8 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
     Params p = base_params(cfg, m, ws, ws_bytes);
     p.pool = pool->w;
     p.scales = pool->s;
+    p.slot_of = pool->slot_of;
+    p.n_slots = pool->n_slots;
     p.w_router = w_router;
     p.bias = bias;
     p.out = out;
@@ -563,6 +581,8 @@ moe_status moe_layer_ex(const moe_config* cfg, const moe_pool* pool, const float
         Params q = base_params(cfg, m, ws, ws_bytes, true);
         q.pool = p.pool;
         q.scales = p.scales;
+        q.slot_of = p.slot_of;
+        q.n_slots = p.n_slots;
         q.w_router = p.w_router;
         q.bias = p.bias;
         q.out = p.out;

@@ -169,6 +169,8 @@ struct Params {
     unsigned long long wait_ns; // bound of the decode kernel's device-side waits (its slot waits: twice this)
     int skip_h_task;            // testing: the one-token decode leaves this task's h unwritten (-1 = none)
     float topp;                 // TOPK/TOPP truncation of the router (0 or 1 = off)
+    const int32_t* slot_of;     // HBM expert cache: expert -> blob slot of `pool` (nullptr: the expert's index)
+    int n_slots;                // with slot_of: the blobs `pool` holds
     const float* w_router;
     const float* bias;
     float* out;
@@ -288,6 +290,11 @@ __device__ __forceinline__ float topp_keep(float topp, int k, float ssum, float 
     kept = lane < k && (lane == 0 || cex < thr);
     const int m = __popc(__ballot_sync(0xffffffffu, kept));
     return __shfl_sync(0xffffffffu, cin, m - 1);
+}
+// The blob of `pool` that holds expert e: its own index, or its slot in an
+// HBM expert cache (every expert a call selects is resident).
+__device__ __forceinline__ int blob_slot(const Params& p, int e, int site) {
+    return p.slot_of ? idx_in(p.ws.hdr, __ldg(p.slot_of + e), 0, p.n_slots, site) : e;
 }
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;

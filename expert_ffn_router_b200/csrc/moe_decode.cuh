@@ -80,7 +80,8 @@ struct DecPlan {
 constexpr int kDecRRMaxRows = 44;
 
 constexpr int kDecRRMaxTasks = kDecMaxK + 1;  // tasks of a single token (row-range down)
-constexpr int kDecRRChunks = 3;  // row-range: 16-byte chunks of the tasks' codes each consumer thread stages
+constexpr int kDecRRChunks = 3;
+constexpr int kDecSlotCache = 260;  // experts (+ shared) whose cache slot the kernel keeps in shared memory  // row-range: 16-byte chunks of the tasks' codes each consumer thread stages
 
 // Shared control block of the kernel, sized for TM tokens.
 template <int TM>
@@ -97,7 +98,7 @@ struct DecCtl {
     int xcs[TM];
     int idx[TM][kDecMaxK];
     float w[TM][kDecMaxK];
-    int4 tasks[kTasks];  // (blob, n tokens, -, -)
+    int4 tasks[kTasks];  // (expert, n tokens, blob slot in the pool, -)
     int ttok[kTasks][TM];
     int sorted[TM * kDecMaxK];    // assignment ids by (expert, token, slot)
     int sorted_e[TM * kDecMaxK];  // their experts
@@ -109,6 +110,7 @@ struct DecCtl {
     int redi[kDecConsWarps];
     float part[kDecGroups][kDecWarps][2 * TM];
     float rsh[kDecRRMaxTasks];  // one token: the scale of each task's staged codes
+    int slot_s[kDecSlotCache];  // HBM expert cache: each expert's blob slot (E + shared <= kDecSlotCache)
 };
 
 // --- consumer reductions over all consumer warps (named barrier 1) ---------
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         C.epoch = __ldcg(&hdr->epoch);
         for (int g = 0; g < kDecGroups; ++g) C.hq_task[g] = -1;
         if (HS) {  // the shared task (task 0): every token, known before any routing
-            C.tasks[0] = make_int4(E, T, 0, 0);
+            C.tasks[0] = make_int4(E, T, E, 0);  // (a cached pool's slot is filled in below)
             for (int t = 0; t < T; ++t) C.ttok[0][t] = t * S + k;
         }
     }
@@ -387,13 +389,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 ++pr;
             }
         };
-        const int n_blobs = E + HS;
-        auto issue_gu = [&](int blob, int j) {
+        const int n_blobs = p.slot_of ? p.n_slots : E + HS;  // blobs the pool holds
+        // the shared expert's blob (its slot in a cached pool, looked up here:
+        // the producer issues the shared rows before the routing)
+        const int sh_slot = blob_slot(p, E, 610);
+        auto issue_gu = [&](int e, int blob, int j) {  // expert e (its scales), in pool blob `blob`
             blob = idx_in(hdr, blob, 0, n_blobs, 611);  // never copy outside the pool, whatever happened
+            e = idx_in(hdr, e, 0, E + HS, 609);
             const int r0 = j * kDecWarps, rows = min(kDecWarps, f - r0);  // f % 8 == 0: rows == 8
             const uint32_t bytes = (uint32_t)rows * rb_gu;
             const uint8_t* base = p.pool + (size_t)blob * p.blob_bytes;
-            const float* sc = p.scales + (size_t)blob * p.scale_rows;
+            const float* sc = p.scales + (size_t)e * p.scale_rows;
             uint64_t* bar = &C.full[ps];
             uint8_t* dst = take(2 * bytes + 2 * rows * 4);
             bulk_g2s(dst, base + (size_t)r0 * rb_gu, bytes, bar);
@@ -441,7 +447,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             }
             const bool tasks_inner = ph == 1 && rmaj;
             for (long long g = 0; g < n_units; ++g) {
-                issue_gu(sh_blob >= 0 ? sh_blob : C.tasks[ti].x, j);
+                if (sh_blob >= 0)
+                    issue_gu(sh_blob, sh_slot, j);
+                else
+                    issue_gu(C.tasks[ti].x, C.tasks[ti].z, j);
                 if (tasks_inner) {
                     if (++ti == n_tasks) {
                         ti = HS;
@@ -464,12 +473,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             const int rot = pl.dn_rot ? c % n_rr : 0;  // the CTA's task order (so the CTAs read different matrices)
             for (int i = 0; i < n_rr; ++i) {
                 const int ti = i + rot < n_rr ? i + rot : i + rot - n_rr;
-                const int blob = idx_in(hdr, C.tasks[ti].x, 0, n_blobs, 612);
+                const int blob = idx_in(hdr, C.tasks[ti].z, 0, n_blobs, 612);
+                const int ex = idx_in(hdr, C.tasks[ti].x, 0, E + HS, 608);
                 const uint32_t wb = (uint32_t)rr_rows * rb_dn;
                 uint8_t* dst = take(wb + (uint32_t)rr_rows * 4);
                 bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)rr_lo * rb_dn, wb,
                          &C.full[ps]);
-                bulk_g2s(dst + pl.wbytes, p.scales + (size_t)blob * p.scale_rows + 2 * f + rr_lo, (uint32_t)rr_rows * 4,
+                bulk_g2s(dst + pl.wbytes, p.scales + (size_t)ex * p.scale_rows + 2 * f + rr_lo, (uint32_t)rr_rows * 4,
                          &C.full[ps]);
                 advance();
             }
@@ -478,14 +488,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             const long long lo = c * Nd / G, hi = (c + 1) * Nd / G;
             int ti = (int)(lo / pl.nu_dn), j = (int)(lo % pl.nu_dn);
             for (long long g = lo; g < hi; ++g) {
-                const int blob = idx_in(hdr, C.tasks[ti].x, 0, n_blobs, 612);
+                const int blob = idx_in(hdr, C.tasks[ti].z, 0, n_blobs, 612);
+                const int ex = idx_in(hdr, C.tasks[ti].x, 0, E + HS, 608);
                 const int r0 = j * pl.rd, rows = min(pl.rd, d - r0);  // multiples of 8
                 const uint32_t bytes = (uint32_t)rows * rb_dn;
                 uint64_t* bar = &C.full[ps];
                 uint8_t* dst = take(bytes + rows * 4);
                 bulk_g2s(dst, p.pool + (size_t)blob * p.blob_bytes + 2 * (size_t)f * rb_gu + (size_t)r0 * rb_dn, bytes,
                          bar);
-                bulk_g2s(dst + pl.wbytes, p.scales + (size_t)blob * p.scale_rows + 2 * f + r0, rows * 4, bar);
+                bulk_g2s(dst + pl.wbytes, p.scales + (size_t)ex * p.scale_rows + 2 * f + r0, rows * 4, bar);
                 advance();
                 if (++j == pl.nu_dn) {
                     j = 0;
@@ -523,6 +534,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
     // ---- 1. the router bias into shared memory (the router reads x as given) ----
     if (E <= kDecBiasCache)
         for (int e = ctid; e < E; e += kDecCons) C.bias_s[e] = __ldg(p.bias + e);
+    // an HBM expert cache: every expert's slot (the producer reads the shared
+    // task's slot only after the routing is published to it)
+    if (p.slot_of) {
+        if (E + HS <= kDecSlotCache)
+            for (int e = ctid; e < E + HS; e += kDecCons) C.slot_s[e] = blob_slot(p, e, 607);
+        if (HS && ctid == 0) C.tasks[0].z = blob_slot(p, E, 607);
+    }
     named_sync(kDecBar, kDecCons);  // the bias cache is filled
 
     // unit index (identical sequence to the producer's) and its ring slot and
@@ -683,6 +701,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
         }
     }
 
+    // the pool blob of expert e (its own index, or its HBM cache slot)
+    auto slot_e = [&](int e) -> int {
+        if (!p.slot_of) return e;
+        return E + HS <= kDecSlotCache ? C.slot_s[e] : blob_slot(p, e, 606);
+    };
+
+    // One token: the h rows of the call are preset to "not written" before the
+    // grid barrier by other CTAs, so an h value computed before the barrier
+    // (the first shared-expert unit) is held in a register and stored once
+    // the barrier has passed -- stored earlier, a CTA that presets later could
+    // overwrite it.
+    bool defer_h = rowrange;
+    float h_held = 0.0f;
+    float* h_held_at = nullptr;
+
     // ---- per-warp gate/up bookkeeping ----
     // Rows finished per task are counted in registers and published once, at
     // the end of the gate/up phase: a fence and an atomic with a returned
@@ -819,8 +852,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                         const float uu = __fmul_rn((float)Uv, __fmul_rn(su, t_sx[i]));
                         const float h = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), uu);
                         // (the h-skip test hook exists only on the row-range path)
-                        if (TM > 1 || ND == 0 || cur_task != p.skip_h_task)
-                            st_relaxed_f32(p.ws.h + (size_t)t_asg[i] * f + r, h);
+                        if (TM > 1 || ND == 0 || cur_task != p.skip_h_task) {
+                            float* dst = p.ws.h + (size_t)t_asg[i] * f + r;
+                            if (defer_h) {  // before the grid barrier: held until it has passed
+                                h_held = h;
+                                h_held_at = dst;
+                            } else {
+                                st_relaxed_f32(dst, h);
+                            }
+                        }
                         amax[i] = fmaxf(amax[i], fabsf(h));
                     }
                 }
@@ -848,6 +888,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
             if (ctid == 0) flag_wait_bounded(&hdr->b1_gen, epoch + 1, hdr, 300, p.wait_ns);
             named_sync(kDecBar, kDecCons);
             if (ctid == 0) DEC_TRACE(4);
+            defer_h = false;
+            if (h_held_at) st_relaxed_f32(h_held_at, h_held);  // every preset of the call is ordered before this
             if (c == 0 && ctid == 0) hdr->epoch = epoch + 1;
             if (warp < T) {
                 int my_e;
@@ -884,7 +926,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                     const bool kept = e != 0x7fffffff;
                     if (kept) {
                         C.ttok[HS + rank][0] = lane;  // assignment id: token 0, slot lane
-                        C.tasks[HS + rank] = make_int4(e, 1, 0, 0);
+                        C.tasks[HS + rank] = make_int4(e, 1, slot_e(e), 0);
                     }
                     const int m = __popc(__ballot_sync(kFull, kept));
                     if (lane == 0) C.n_tasks = HS + m;
@@ -913,7 +955,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const Params p, const
                 }
                 for (int q = 0; q < A; ++q) n += C.sorted_e[q] == ea;
                 C.ttok[HS + tq][rank] = (a / k) * S + (a % k);
-                if (rank == 0) C.tasks[HS + tq] = make_int4(ea, n, 0, 0);
+                if (rank == 0) C.tasks[HS + tq] = make_int4(ea, n, slot_e(ea), 0);
                 if (ctid == A - 1 || C.sorted_e[ctid + 1] == E) C.n_tasks = HS + tq + 1;  // the last kept one
             }
             named_sync(kDecBar, kDecCons);

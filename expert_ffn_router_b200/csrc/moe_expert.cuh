@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(kThreads) k_gate_up(const Params p) {
             if (tid == 0) s_n = nn;
         }
         const int bx = idx_in(p.ws.hdr, task.x, 0, p.m.E + p.m.has_shared, 624);
-        const uint8_t* blob = p.pool + (size_t)bx * p.blob_bytes;
+        const uint8_t* blob = p.pool + (size_t)blob_slot(p, bx, 625) * p.blob_bytes;
         const float* sc = p.scales + (size_t)bx * p.scale_rows;
         float amax[CH];
 #pragma unroll
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kThreads) k_down(const Params p) {
             __syncthreads();
         }
         const int bx = idx_in(p.ws.hdr, task.x, 0, p.m.E + p.m.has_shared, 634);
-        const uint8_t* wd = p.pool + (size_t)bx * p.blob_bytes + 2 * (size_t)f * (d * WB / 8);
+        const uint8_t* wd = p.pool + (size_t)blob_slot(p, bx, 635) * p.blob_bytes + 2 * (size_t)f * (d * WB / 8);
         const float* sd = p.scales + (size_t)bx * p.scale_rows + 2 * f;
         const int r0 = rb * RB + warp * RPW;
         uint4 wv[RPW][NCL];

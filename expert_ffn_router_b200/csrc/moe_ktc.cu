@@ -72,7 +72,7 @@ static cudaError_t launch_tc_t(const Params& p, const CUtensorMap& tm, int nt_ma
 }
 
 cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_t s) {
-    const int E1 = p.m.E + p.m.has_shared;
+    const int E1 = p.slot_of ? p.n_slots : p.m.E + p.m.has_shared;  // blobs the pool holds
     CUtensorMap tm;
     const int wb = p.m.wb;
     cudaError_t e;

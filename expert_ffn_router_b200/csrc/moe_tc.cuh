@@ -195,8 +195,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int4 task = p.ws.tasks[ti];
                 const int npad = tc_npad(idx_in(hdr, task.z, 1, kTcNT + 1, 641));
                 const uint32_t bbytes = (uint32_t)npad * KC;
-                const int bx = idx_in(hdr, task.x, 0, p.m.E + p.m.has_shared, 642);
-                int y0, y1;
+                const int bx = blob_slot(p, idx_in(hdr, task.x, 0, p.m.E + p.m.has_shared, 642), 649);
+                int y0, y1;  // rows of the pool map (the task's blob: its expert, or its cache slot)
                 if (EPI == 0) {
                     y0 = bx * 3 * f + rb * 128;
                     y1 = y0 + f;

@@ -99,15 +99,24 @@ typedef struct {
     float topp;
 } moe_config;
 
-/* One layer's experts, resident in device memory, canonical layout.
+/* One layer's experts in device memory, canonical layout.
  *  w: E + has_shared blobs of 3*d*f*wbits/8 bytes each, expert e at offset
  *     e * blob_bytes, the shared expert last.  A blob is
  *     [gate f x d | up f x d | down d x f], each matrix row-major by output
  *     row, codes packed as above ("adjacent matrices stored together").
- *  s: fp32 [E + has_shared][f + f + d] per-output-row scales, same order. */
+ *  s: fp32 [E + has_shared][f + f + d] per-output-row scales, same order
+ *     (always every expert's: 10 KB each at the GLM-5.2 shape).
+ *  slot_of: NULL, or an HBM expert cache's slot table (moe_cache below):
+ *     device int32 [E + has_shared]; then w holds n_slots blobs and expert e's
+ *     blob is at w + slot_of[e] * blob_bytes.  Every expert a call selects
+ *     must be resident (moe_cache_fetch); an index outside [0, n_slots) is
+ *     clamped (and recorded as MOE_EDEVICE by the bounds-checked build).
+ *  n_slots: the blobs w holds when slot_of is set. */
 typedef struct {
     const uint8_t* w;
     const float* s;
+    const int32_t* slot_of;
+    int32_t n_slots;
 } moe_pool;
 
 /* Bytes of workspace the calls below need for up to max_tokens tokens. */
@@ -259,6 +268,50 @@ MOE_API moe_status moe_rmsnorm(const void* x, moe_dtype dtype, int32_t T, int32_
  * error).  Synchronises `stream` first.  *info (optional) receives a detail
  * word. */
 MOE_API moe_status moe_poll_status(const void* ws, int32_t* info, moe_stream_t stream);
+
+/* HBM expert cache with host-memory overflow, one per layer: the layer's
+ * full pool stays in pinned host memory, n_slots blobs of it are resident in
+ * device memory, and moe_cache_fetch makes the experts a call selects
+ * resident before the call runs, evicting the least recently used others
+ * (the pages' per-layer LRU of experts with readahead -- agentlenshq,
+ * "ロードメカニズム"; remio.ai, the async I/O pool paragraph -- moved one tier
+ * up: host RAM behind HBM instead of disk behind RAM).  All memory is the
+ * caller's:
+ *  host_w: pinned host memory, the layer's E + has_shared blobs (canonical
+ *          layout, as moe_pool.w);
+ *  slots: device memory, n_slots blobs (16-byte aligned);
+ *  slot_of: device int32 [E + has_shared], written by the calls below;
+ *  state: host memory of moe_cache_state_bytes(cfg, n_slots) bytes (the LRU
+ *         book-keeping);
+ *  n_slots: >= the distinct experts of one call (+ the shared expert).
+ * Use: moe_cache_init once; per call: route (moe_route), copy the indices to
+ * the host, moe_cache_fetch, then moe_layer with the pool {slots, scales,
+ * slot_of, n_slots} on the same stream (the layer routes again and finds the
+ * same experts).  The shared expert is fetched at init and never evicted. */
+typedef struct {
+    const uint8_t* host_w;
+    uint8_t* slots;
+    int32_t* slot_of;
+    void* state;
+    int32_t n_slots;
+} moe_cache;
+typedef struct {
+    int64_t hits;    /* experts a fetch found resident */
+    int64_t misses;  /* experts it copied in */
+    int64_t bytes;   /* host -> device bytes it issued */
+} moe_cache_stats;
+MOE_API size_t moe_cache_state_bytes(const moe_config* cfg, int32_t n_slots);
+/* Empties the cache, copies the shared expert in (slot 0) and writes slot_of
+ * (-1 for every other expert).  Host errors return synchronously. */
+MOE_API moe_status moe_cache_init(const moe_config* cfg, moe_cache* cache, moe_stream_t stream);
+/* Makes every expert in idx (host int32 [T][top_k], -1 entries skipped)
+ * resident: a hit refreshes the expert's use; a miss takes a free slot or
+ * the least recently used slot whose expert this call does not select, and
+ * issues one cudaMemcpyAsync of its blob on `stream`; then one copy of the
+ * updated slot table.  MOE_ENOSPACE if n_slots cannot hold the call's
+ * experts.  stats (nullable) receives this call's counts. */
+MOE_API moe_status moe_cache_fetch(const moe_config* cfg, moe_cache* cache, const int32_t* idx, int32_t T,
+                                   moe_stream_t stream, moe_cache_stats* stats);
 
 MOE_API const char* moe_status_string(moe_status status);
 MOE_API const char* moe_last_error(void);

@@ -114,3 +114,27 @@ def test_layer_opts_rejects_negative_test_fields():
     st = L.moe_layer_ex(ctypes.byref(c), ctypes.byref(pool), FAKE, FAKE, FAKE, 0, 4, FAKE, 0, None, None, FAKE,
                         1 << 40, None, ctypes.byref(o))
     assert st == M.MOE_EINVAL
+
+
+def test_cache_entry_points_validate_on_the_host():
+    c = good_cfg()
+    assert L.moe_cache_state_bytes(ctypes.byref(c), 0) == 0
+    n4 = L.moe_cache_state_bytes(ctypes.byref(c), 4)
+    assert n4 > L.moe_cache_state_bytes(ctypes.byref(c), 2) > 0
+    cache = M.MoeCache(FAKE, FAKE, FAKE, FAKE, 1)  # one slot cannot hold the shared expert and another
+    assert L.moe_cache_init(ctypes.byref(c), ctypes.byref(cache), None) == M.MOE_EINVAL
+    cache = M.MoeCache(None, FAKE, FAKE, FAKE, 4)
+    assert L.moe_cache_init(ctypes.byref(c), ctypes.byref(cache), None) == M.MOE_EINVAL
+    cache = M.MoeCache(FAKE, FAKE + 4, FAKE, FAKE, 4)  # slots not 16-byte aligned
+    assert L.moe_cache_init(ctypes.byref(c), ctypes.byref(cache), None) == M.MOE_EALIGN
+    # a fetch before init is refused (the state's header does not match)
+    state = (ctypes.c_uint64 * (n4 // 8 + 1))()
+    cache = M.MoeCache(FAKE, FAKE, FAKE, ctypes.addressof(state), 4)
+    idx = (ctypes.c_int32 * 2)(0, 1)
+    assert L.moe_cache_fetch(ctypes.byref(c), ctypes.byref(cache), ctypes.addressof(idx), 1, None, None) == \
+        M.MOE_EINVAL
+    # a pool with a slot table must say how many blobs it holds
+    pool = M.MoePool(FAKE, FAKE, FAKE, 0)
+    st = L.moe_layer(ctypes.byref(c), ctypes.byref(pool), FAKE, FAKE, FAKE, 0, 4, FAKE, 0, None, None, FAKE,
+                     1 << 40, None)
+    assert st == M.MOE_EINVAL
