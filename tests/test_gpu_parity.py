@@ -389,3 +389,32 @@ def test_layer_one_token_small_pools(name):
     M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(x), acc, ws, accumulate=True)
     assert_ok(ws)
     np.testing.assert_allclose(acc.cpu().numpy(), (base + out).cpu().numpy(), rtol=1e-6, atol=1e-5)
+
+
+@pytest.mark.parametrize("E", [8, 16, 24])
+def test_layer_decode_few_experts_many_calls(E):
+    """One token at the GLM-5.2 expert shape with pools of few experts: most
+    CTAs own no router row and reach their first shared-expert unit right
+    after quantising, while other CTAs still preset the call's h rows; the h
+    values of that unit are stored only after the grid barrier, so none is
+    erased by a late preset (which made the hand-off's poll run out).  60
+    calls, every status OK, and each token's output against the oracle."""
+    wl = W.workload(1).replace(name=f"glm_few_e{E}", n_experts=E, top_k=min(8, E))
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    cfg = cfg_of(wl)
+    pool = M.make_pool(dl.pool_w, dl.pool_s)
+    ws = M.workspace(cfg, 1)
+    outs, idxs, xs = {}, {}, [x_host(wl, s) for s in range(3)]
+    for it in range(60):
+        out = torch.empty(1, wl.d, device="cuda")
+        idx = torch.empty(1, wl.top_k, dtype=torch.int32, device="cuda")
+        M.moe_layer(cfg, pool, dl.w_router, dl.bias, to_dev(xs[it % 3]), out, ws, topk_idx_out=idx)
+        torch.cuda.synchronize()
+        assert_ok(ws)
+        if it % 3 in outs:
+            assert torch.equal(out, outs[it % 3])
+        else:
+            outs[it % 3], idxs[it % 3] = out, idx.cpu().numpy()
+    for s_ in range(3):
+        compare_layer(wl, L, xs[s_], outs[s_], idxs[s_])
