@@ -44,7 +44,9 @@
  * as written.
  *
  * Packing [reading]: codes are two's complement, low bits first within a byte:
- * int4 byte = c0 | c1 << 4; int2 byte = c0 | c1 << 2 | c2 << 4 | c3 << 6.
+ * int4 byte = c0 | c1 << 4; int2 byte = c0 | c1 << 2 | c2 << 4 | c3 << 6;
+ * int8 experts (the "expert@8-bit" banner of the takumi3488 run log): one
+ * code per byte, [-128, 127].
  * Expert blob [reading of "adjacent matrices stored together", remio.ai
  * analysis, the dedupe paragraph]: [gate f x d | up f x d | down d x f], each
  * matrix row-major by output row; scales [gate f | up f | down d].
@@ -79,7 +81,8 @@ void oracle_set_num_threads(int n) {
 #endif
 }
 
-/* Code i of a packed row: wbits in {2, 4}, two's complement, low bits first. */
+/* Code i of a packed row: wbits in {2, 4, 8}, two's complement, low bits first
+ * (int8: one code per byte). */
 static inline int code_at(const uint8_t* row, int wbits, int64_t i) {
     int per_byte = 8 / wbits;
     int shift = (int)(i % per_byte) * wbits;
@@ -88,13 +91,13 @@ static inline int code_at(const uint8_t* row, int wbits, int64_t i) {
 }
 
 int oracle_unpack(int wbits, const uint8_t* src, int64_t n, int8_t* dst) {
-    if ((wbits != 2 && wbits != 4) || !src || !dst || n < 0) return ORACLE_EINVAL;
+    if ((wbits != 2 && wbits != 4 && wbits != 8) || !src || !dst || n < 0) return ORACLE_EINVAL;
     for (int64_t i = 0; i < n; ++i) dst[i] = (int8_t)code_at(src, wbits, i);
     return ORACLE_OK;
 }
 
 int oracle_pack(int wbits, const int8_t* src, int64_t n, uint8_t* dst) {
-    if ((wbits != 2 && wbits != 4) || !src || !dst || n < 0) return ORACLE_EINVAL;
+    if ((wbits != 2 && wbits != 4 && wbits != 8) || !src || !dst || n < 0) return ORACLE_EINVAL;
     int per_byte = 8 / wbits;
     if (n % per_byte) return ORACLE_EINVAL;
     int lo = -(1 << (wbits - 1)), hi = (1 << (wbits - 1)) - 1;
@@ -224,7 +227,7 @@ static int fits_i32(int64_t v) { return v >= INT32_MIN && v <= INT32_MAX; }
  * hq int8 [T][f], sh fp32 [T] -> acc_d int32 [T][d] (nullable), y fp64 [T][d]. */
 int oracle_down(int d, int f, int wbits, const uint8_t* blob, const float* sc, const int8_t* hq,
                 const float* sh, int T, int32_t* acc_d, double* y) {
-    if ((wbits != 2 && wbits != 4) || !blob || !sc || !hq || !sh || !y || d <= 0 || f <= 0 || T < 0)
+    if ((wbits != 2 && wbits != 4 && wbits != 8) || !blob || !sc || !hq || !sh || !y || d <= 0 || f <= 0 || T < 0)
         return ORACLE_EINVAL;
     const int64_t row_gu = (int64_t)d * wbits / 8, row_dn = (int64_t)f * wbits / 8;
     const uint8_t* wd = blob + 2 * (int64_t)f * row_gu;
@@ -249,7 +252,7 @@ int oracle_down(int d, int f, int wbits, const uint8_t* blob, const float* sc, c
 int oracle_expert(int d, int f, int wbits, const uint8_t* blob, const float* sc, const int8_t* xq,
                   const float* sx, int T, int32_t* acc_gu, float* h_out, int8_t* hq_out,
                   float* sh_out, int32_t* acc_d, double* y) {
-    if ((wbits != 2 && wbits != 4) || !blob || !sc || !xq || !sx || !y || d <= 0 || f <= 0 || T < 0)
+    if ((wbits != 2 && wbits != 4 && wbits != 8) || !blob || !sc || !xq || !sx || !y || d <= 0 || f <= 0 || T < 0)
         return ORACLE_EINVAL;
     const int64_t row_gu = (int64_t)d * wbits / 8;
     const uint8_t* wg = blob;

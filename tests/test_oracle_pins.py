@@ -41,7 +41,7 @@ def unpack_np(wbits, packed, n):
 # --------------------------------------------------------------------------
 # packing
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("wbits", [4, 2])
+@pytest.mark.parametrize("wbits", [4, 2, 8])
 def test_pack_unpack_roundtrip_every_code_every_position(wbits):
     lo, hi = -(1 << (wbits - 1)), (1 << (wbits - 1)) - 1
     per = 8 // wbits
@@ -62,6 +62,8 @@ def test_unpack_hand_bytes():
     np.testing.assert_array_equal(O.unpack(4, np.array([0x8F, 0x71], np.uint8), 4), [-1, -8, 1, 7])
     # int2: 0xE4 = 0b11_10_01_00 -> crumbs low first: 0, 1, -2, -1
     np.testing.assert_array_equal(O.unpack(2, np.array([0xE4], np.uint8), 4), [0, 1, -2, -1])
+    # int8: one two's-complement code per byte
+    np.testing.assert_array_equal(O.unpack(8, np.array([0x80, 0xFF, 0x00, 0x7F], np.uint8), 4), [-128, -1, 0, 127])
 
 
 # --------------------------------------------------------------------------
@@ -166,7 +168,7 @@ def test_router_exact_ties_pick_lower_index():
 # --------------------------------------------------------------------------
 # a3/a4 integer dots: exact identities against int64 matmul of unpacked codes
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("wbits,d,f,T", [(4, 64, 32, 3), (2, 64, 48, 2), (4, 96, 40, 1)])
+@pytest.mark.parametrize("wbits,d,f,T", [(4, 64, 32, 3), (2, 64, 48, 2), (4, 96, 40, 1), (8, 64, 32, 2)])
 def test_expert_integer_identities(wbits, d, f, T):
     rng = np.random.default_rng(wbits * 1000 + d)
     blob = rng.integers(0, 256, 3 * d * f * wbits // 8, dtype=np.uint8)
