@@ -90,7 +90,9 @@ static int round_ncl(int ncl, bool down) {
     if (ncl <= 2) return 2;
     if (ncl <= 4) return 4;
     if (!down && ncl <= 6) return 6;
-    return 8;
+    if (ncl <= 8) return 8;
+    if (ncl <= 12) return 12;  // rows above 4 KB: int8 experts only
+    return 16;
 }
 
 ExpertTiling expert_tiling(int d, int f, int wb) {
@@ -112,7 +114,7 @@ moe_status check_cfg(const moe_config* c) {
     if (!c) return fail(MOE_EINVAL, "cfg is NULL");
     if (c->d <= 0 || c->f <= 0 || c->d > 8192 || c->f > 8192)
         return fail(MOE_EINVAL, "d and f must be in [1, 8192]");
-    if (c->wbits != 4 && c->wbits != 2) return fail(MOE_EINVAL, "wbits must be 4 or 2");
+    if (c->wbits != 4 && c->wbits != 2 && c->wbits != 8) return fail(MOE_EINVAL, "wbits must be 4, 2 or 8");
     if ((c->d * c->wbits / 8) % 16 || (c->f * c->wbits / 8) % 16 || (c->d * c->wbits) % 8 || (c->f * c->wbits) % 8)
         return fail(MOE_EINVAL, "d*wbits/8 and f*wbits/8 must be multiples of 16 bytes");
     if (c->n_experts < 1 || c->n_experts > 1024) return fail(MOE_EINVAL, "n_experts must be in [1, 1024]");

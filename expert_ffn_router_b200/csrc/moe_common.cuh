@@ -427,7 +427,12 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, int v[8]) {
                  : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// 16 / 32 consecutive 32-bit TMEM columns of this thread's lane <- registers.
+// 8 / 16 / 32 consecutive 32-bit TMEM columns of this thread's lane <- registers.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t v[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t v[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -579,9 +584,10 @@ static __device__ int block_exscan(int* a, int n, int* red) {
 
 // ---------------------------------------------------------------------------
 // Activation staging layout.  A 16-byte chunk of packed weights holds 32 int4
-// codes (or 64 int2 codes).  The dot kernels split each weight word into
-// byte lanes with one mask (offset-binary codes u = c + 8 or c + 2), so the
-// int8 activations are stored per chunk in the matching byte order:
+// codes (or 64 int2, or 16 int8 codes).  The dot kernels split each weight
+// word into byte lanes with one mask (offset-binary codes u = c + 8, c + 2 or
+// c + 128), so the int8 activations are stored per chunk in the matching byte
+// order (int8 weights: the natural order):
 //  int4: per 8 columns, word E = (x0,x2,x4,x6) then word O = (x1,x3,x5,x7);
 //        sub-array s (s = 0, 1) of a chunk holds columns 16s .. 16s+15.
 //  int2: per 16 columns, words P_m = (x_m, x_{m+4}, x_{m+8}, x_{m+12}),
@@ -592,7 +598,9 @@ static __device__ int block_exscan(int* a, int n, int* red) {
 template <int WB>
 __device__ __forceinline__ uint4 permute16(uint4 n) {
     uint4 r;
-    if (WB == 4) {
+    if (WB == 8) {  // one code per byte: the natural order
+        r = n;
+    } else if (WB == 4) {
         r.x = __byte_perm(n.x, n.y, 0x6420);
         r.y = __byte_perm(n.x, n.y, 0x7531);
         r.z = __byte_perm(n.z, n.w, 0x6420);
@@ -639,7 +647,13 @@ __device__ __forceinline__ int stage_row(const int8_t* src, int ncols, uint4* ds
 // Dot of one 16-byte weight chunk with one staged activation chunk.
 template <int WB>
 __device__ __forceinline__ int dot_chunk(const uint4 w, const uint4* xs, int nch, int c, int acc) {
-    if (WB == 4) {
+    if (WB == 8) {  // 16 codes, offset-binary bytes c + 128 by flipping each sign bit
+        const uint4 x0 = xs[c];
+        acc = dp4a_us(w.x ^ 0x80808080u, (int)x0.x, acc);
+        acc = dp4a_us(w.y ^ 0x80808080u, (int)x0.y, acc);
+        acc = dp4a_us(w.z ^ 0x80808080u, (int)x0.z, acc);
+        acc = dp4a_us(w.w ^ 0x80808080u, (int)x0.w, acc);
+    } else if (WB == 4) {
         const uint4 x0 = xs[c], x1 = xs[nch + c];
         const unsigned a = w.x ^ 0x88888888u, b = w.y ^ 0x88888888u;
         const unsigned cc = w.z ^ 0x88888888u, dd = w.w ^ 0x88888888u;
@@ -667,7 +681,7 @@ __device__ __forceinline__ int dot_chunk(const uint4 w, const uint4* xs, int nch
 
 // Offset of the offset-binary codes: sum c*x = sum u*x - kOff * sum x.
 template <int WB>
-__device__ __forceinline__ constexpr int code_offset() { return WB == 4 ? 8 : 2; }
+__device__ __forceinline__ constexpr int code_offset() { return WB == 8 ? 128 : WB == 4 ? 8 : 2; }
 
 // Order-preserving map of a float to an unsigned key (larger float, larger key).
 __device__ __forceinline__ unsigned float_key(float v) {

@@ -80,8 +80,8 @@ struct DecPlan {
 constexpr int kDecRRMaxRows = 44;
 
 constexpr int kDecRRMaxTasks = kDecMaxK + 1;  // tasks of a single token (row-range down)
-constexpr int kDecRRChunks = 3;
-constexpr int kDecSlotCache = 260;  // experts (+ shared) whose cache slot the kernel keeps in shared memory  // row-range: 16-byte chunks of the tasks' codes each consumer thread stages
+constexpr int kDecRRChunks = 3;     // row-range: 16-byte chunks of the tasks' codes each consumer thread stages
+constexpr int kDecSlotCache = 260;  // experts (+ shared) whose cache slot the kernel keeps in shared memory
 
 // Shared control block of the kernel, sized for TM tokens.
 template <int TM>
@@ -151,7 +151,12 @@ __device__ __forceinline__ int grp_sum_int(int v, int* red, int g) {
 // odd weight words) to halve the dependent dp4a chain.
 template <int WB>
 __device__ __forceinline__ void dot_chunk_regs(const uint4 w, const uint4* x, int& a0, int& a1) {
-    if (WB == 4) {
+    if (WB == 8) {  // 16 codes, offset-binary by flipping each sign bit
+        a0 = dp4a_us(w.x ^ 0x80808080u, (int)x[0].x, a0);
+        a1 = dp4a_us(w.y ^ 0x80808080u, (int)x[0].y, a1);
+        a0 = dp4a_us(w.z ^ 0x80808080u, (int)x[0].z, a0);
+        a1 = dp4a_us(w.w ^ 0x80808080u, (int)x[0].w, a1);
+    } else if (WB == 4) {
         const unsigned p = w.x ^ 0x88888888u, q = w.y ^ 0x88888888u;
         const unsigned r = w.z ^ 0x88888888u, t = w.w ^ 0x88888888u;
         a0 = dp4a_us(p & 0x0F0F0F0Fu, (int)x[0].x, a0);

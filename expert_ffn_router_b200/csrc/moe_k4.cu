@@ -22,6 +22,12 @@ static cudaError_t by_ncl(const Params& p, int ncl, cudaStream_t s) {
         case 2: return go4<WB, CH, 2, DBG>(p, s);
         case 4: return go4<WB, CH, 4, DBG>(p, s);
         case 8: return go4<WB, CH, 8, DBG>(p, s);
+        case 12:  // rows of 6 KB and 8 KB: int8 experts only
+            if constexpr (WB == 8) return go4<WB, CH, 12, DBG>(p, s);
+            return cudaErrorInvalidValue;
+        case 16:
+            if constexpr (WB == 8) return go4<WB, CH, 16, DBG>(p, s);
+            return cudaErrorInvalidValue;
         default: return cudaErrorInvalidValue;
     }
 }
@@ -39,6 +45,7 @@ static cudaError_t by_ch(const Params& p, int ncl, bool dbg, cudaStream_t s) {
 }
 
 cudaError_t launch_down(const Params& p, const ExpertTiling& tl, bool dbg, cudaStream_t s) {
+    if (p.m.wb == 8) return by_ch<8>(p, tl.ncl4, dbg, s);
     return p.m.wb == 4 ? by_ch<4>(p, tl.ncl4, dbg, s) : by_ch<2>(p, tl.ncl4, dbg, s);
 }
 

@@ -125,16 +125,19 @@ static cudaError_t by_t(const Params& p, const DecPlan& pl, const void* x, cudaS
 
 // Fully unrolled rows for the GLM-5.2 expert shape (d = 6144, f = 2048):
 // 6 (int4) or 3 (int2) 16-byte chunks per lane of a gate/up row, 2 or 1 of a
-// down row; any other shape takes the runtime loop.
+// down row; any other shape (and int8 experts) takes the runtime loop.
 template <int WB, typename XT>
 static cudaError_t by_shape(const Params& p, const DecPlan& pl, const void* x, cudaStream_t s) {
     const int nch_gu = p.m.d * WB / 8 / 16, nch_dn = p.m.f * WB / 8 / 16;
+    if constexpr (WB == 8) return by_t<WB, 0, 0, XT>(p, pl, x, s);
     constexpr int NG = WB == 4 ? 6 : 3, ND = WB == 4 ? 2 : 1;
     if (nch_gu == 32 * NG && nch_dn == 32 * ND && pl.rd == kDecNQ * kDecWarps) return by_t<WB, NG, ND, XT>(p, pl, x, s);
     return by_t<WB, 0, 0, XT>(p, pl, x, s);
 }
 
 cudaError_t launch_decode(const Params& p, const DecPlan& pl, const void* x, bool bf16, cudaStream_t s) {
+    if (p.m.wb == 8)
+        return bf16 ? by_shape<8, __nv_bfloat16>(p, pl, x, s) : by_shape<8, float>(p, pl, x, s);
     if (p.m.wb == 4)
         return bf16 ? by_shape<4, __nv_bfloat16>(p, pl, x, s) : by_shape<4, float>(p, pl, x, s);
     return bf16 ? by_shape<2, __nv_bfloat16>(p, pl, x, s) : by_shape<2, float>(p, pl, x, s);

@@ -81,6 +81,7 @@ cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_
     else
         e = make_pool_map(&tm, p.pool, (uint64_t)p.m.f * wb / 8, (uint64_t)3 * p.m.d * E1);
     if (e != cudaSuccess) return e;
+    if (wb == 8) return stage == 0 ? launch_tc_t<8, 0>(p, tm, nt_max, s) : launch_tc_t<8, 1>(p, tm, nt_max, s);
     if (wb == 4) return stage == 0 ? launch_tc_t<4, 0>(p, tm, nt_max, s) : launch_tc_t<4, 1>(p, tm, nt_max, s);
     return stage == 0 ? launch_tc_t<2, 0>(p, tm, nt_max, s) : launch_tc_t<2, 1>(p, tm, nt_max, s);
 }
@@ -88,7 +89,8 @@ cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_
 cudaError_t launch_tc_requant(const Params& p, cudaStream_t s) {
     const int grid = (int)std::min<size_t>((tc_rows_bound(p.m) + kWarps - 1) / kWarps,
                                            (size_t)persistent_grid((const void*)k_tc_requant<4>, 0));
-    if (p.m.wb == 4) k_tc_requant<4><<<grid, kThreads, 0, s>>>(p);
+    if (p.m.wb == 8) k_tc_requant<8><<<grid, kThreads, 0, s>>>(p);
+    else if (p.m.wb == 4) k_tc_requant<4><<<grid, kThreads, 0, s>>>(p);
     else k_tc_requant<2><<<grid, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
@@ -99,7 +101,8 @@ cudaError_t launch_tc_gather(const Params& p, const int8_t* src, int ld, int key
     // one warp per padded row; the row count is known on the device only
     const int grid = (int)std::min<size_t>((tc_rows_bound(p.m) + kWarps - 1) / kWarps,
                                            (size_t)persistent_grid((const void*)k_tc_gather<4>, 0));
-    if (p.m.wb == 4) k_tc_gather<4><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
+    if (p.m.wb == 8) k_tc_gather<8><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
+    else if (p.m.wb == 4) k_tc_gather<4><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
     else k_tc_gather<2><<<grid, kThreads, 0, s>>>(p, src, ld, key_div, K, kpad, dst);
     return cudaGetLastError();
 }

@@ -43,7 +43,7 @@
 //                   combine is a separate kernel) or straight to the output.
 // TMEM columns: two accumulator buffers [128 b, 128 b + 128) (tile 0 at
 // +0, tile 1 at +64, N <= 64), then the A buffers from column 256 (2 x KC/4
-// columns each: four for int4, two for int2).  Every wait is bounded
+// columns each: eight buffers for int8, four for int4, two for int2).  Every wait is bounded
 // (kWaitLimitNs); on a timeout the CTA records MOE_ETIMEOUT, lets its copies
 // and MMAs drain and exits.
 #pragma once
@@ -61,11 +61,12 @@ constexpr int kTcEpi = 128;
 constexpr int kTcBox = 128 * 64;               // one A box: 128 rows x 64 packed bytes
 constexpr int kTcSlotA = 2 * kTcBox;           // both tiles of a chunk
 constexpr int kTcMaxSlots = 8;
+constexpr int kTcMaxAB = 8;                    // TMEM A buffers: 256 columns / (2 tiles x KC/4), KC = 64 for int8
 
 // Dynamic shared memory: [slots][control block], slots 1024-byte aligned.
 struct TcCtl {
     uint64_t full[kTcMaxSlots], empty[kTcMaxSlots];
-    uint64_t afull[4], afree[4], accfull[2], accempty[2], drain;
+    uint64_t afull[kTcMaxAB], afree[kTcMaxAB], accfull[2], accempty[2], drain;
     uint32_t tmem_base;
     int asg[kTcNT];
     float sx[kTcNT];
@@ -103,7 +104,18 @@ template <int WB>
 __device__ __forceinline__ void tc_unpack_tile(const uint8_t* box, int row, int hh, uint32_t taddr) {
     const uint8_t* rp = box + row * 64;
     const int sw = (row >> 1) & 3;
-    if (WB == 4) {
+    if (WB == 8) {  // one code per byte: flip each sign bit
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + (((2 * hh + j) ^ sw) << 4));
+            w[4 * j] = v.x ^ 0x80808080u;
+            w[4 * j + 1] = v.y ^ 0x80808080u;
+            w[4 * j + 2] = v.z ^ 0x80808080u;
+            w[4 * j + 3] = v.w ^ 0x80808080u;
+        }
+        tmem_st8(taddr, w);
+    } else if (WB == 4) {
         uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -146,6 +158,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int ACOLS = KC / 4;           // TMEM columns of one tile's A chunk
     constexpr int KSTEPS = KC / 32;
     constexpr int NAB = 256 / (2 * ACOLS);  // TMEM A buffers
+    static_assert(NAB <= kTcMaxAB, "TcCtl holds kTcMaxAB A-buffer barriers");
     constexpr int OFF = code_offset<WB>();
     extern __shared__ uint8_t tc_raw[];
     uint8_t* base = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023u)) & 1023u);

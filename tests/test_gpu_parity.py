@@ -30,6 +30,9 @@ SMALL = {
     "ragged_int2_T2": W.workload(0).replace(name="ragged_int2", d=1088, f=320, n_experts=24, top_k=5, T=2,
                                             wbits=2),
     "wide_k": W.workload(0).replace(name="wide_k", d=256, f=96, n_experts=64, top_k=32, T=7),
+    "ragged_int8": W.workload(0).replace(name="ragged_int8", d=1056, f=352, n_experts=24, top_k=5, T=13, wbits=8),
+    "ragged_int8_T2": W.workload(0).replace(name="ragged_int8", d=1056, f=352, n_experts=24, top_k=5, T=2,
+                                            wbits=8),
 }
 PATHS = {"auto": M.MOE_PATH_AUTO, "multi": M.MOE_PATH_MULTI, "decode": M.MOE_PATH_DECODE}
 
@@ -40,7 +43,7 @@ def auto_path(T):
     return M.MOE_PATH_DECODE if T <= 2 else M.MOE_PATH_TC
 
 # One-token decode on small pools of d = 2048 (the decode kernel's runtime-loop
-# rows): int4 and int2 rows, no shared expert, E > 256 (its shared-memory
+# rows): int4, int2 and int8 rows, no shared expert, E > 256 (its shared-memory
 # top-k) and k = 32.
 SINGLE = {
     "s1_int4": W.workload(0).replace(name="s1_int4", d=2048, f=1024, n_experts=16, top_k=4, T=1, x_dtype="bf16"),
@@ -50,6 +53,8 @@ SINGLE = {
                                           has_shared=0),
     "s1_E512": W.workload(0).replace(name="s1_E512", d=2048, f=1024, n_experts=512, top_k=8, T=1),
     "s1_k32": W.workload(0).replace(name="s1_k32", d=2048, f=1024, n_experts=64, top_k=32, T=1),
+    "s1_int8": W.workload(0).replace(name="s1_int8", d=2048, f=1024, n_experts=16, top_k=4, T=1, wbits=8,
+                                     x_dtype="bf16"),
 }
 
 
@@ -117,7 +122,8 @@ def test_route_full_size(T):
 
 
 EXPERT_CASES = [("tiny", 4, 1), ("ragged_int4", 9, 1), ("ragged_int4", 3, -1), ("ragged_int2", 11, 2),
-                ("full_int4", 1, 7), ("full_int4", 9, -1), ("full_int2", 3, 5)]
+                ("full_int4", 1, 7), ("full_int4", 9, -1), ("full_int2", 3, 5), ("ragged_int8", 9, 1),
+                ("ragged_int8", 3, -1)]
 
 
 @pytest.mark.parametrize("name,T,expert", EXPERT_CASES)

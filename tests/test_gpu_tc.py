@@ -5,9 +5,10 @@ Forced with moe_config.tc_min_tokens = 1 (or the layer's MOE_PATH_TC).  Cases
 span: padded token counts of 8 and 16 and a multiple of 16, tasks split at 64
 tokens (130, 160, 300 tokens of one expert), ragged K (d = 1056: the last
 128-column chunk is partly outside the row; f = 320 with int2: 256-column
-chunks), ragged rows (f = 352: the last 128-row tile is partly another
-matrix's rows), int4 and int2, routed and shared experts, and the full
-d = 6144, f = 2048 shapes.  Integer accumulators must be bit-exact.
+chunks; int8 rows: 64-column chunks), ragged rows (f = 352: the last 128-row
+tile is partly another matrix's rows), int8, int4 and int2 weights, routed and
+shared experts, and the full d = 6144, f = 2048 shapes.  Integer accumulators
+must be bit-exact.
 """
 import numpy as np
 import pytest
@@ -28,7 +29,7 @@ def cfg_tc(wl, thr=1):
 
 TC_EXPERT_CASES = [("tiny", 4, 1), ("tiny", 32, -1), ("ragged_int4", 9, 1), ("ragged_int4", 130, -1),
                    ("ragged_int2", 11, 2), ("ragged_int2", 40, -1), ("full_int4", 1, 7), ("full_int4", 160, -1),
-                   ("full_int4", 300, 3), ("full_int2", 24, 5)]
+                   ("full_int4", 300, 3), ("full_int2", 24, 5), ("ragged_int8", 9, 1), ("ragged_int8", 40, -1)]
 
 
 def single_expert_pool(wl, e):
