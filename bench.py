@@ -61,6 +61,8 @@ def parse(argv=None):
                          "(moe_config.topp; fewer experts per token)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="supplementary case: the workload with this many tokens per step (e.g. prefill at 8192)")
+    ap.add_argument("--wbits", type=int, choices=[2, 4, 8], default=0,
+                    help="supplementary case: the workload with expert codes of this width (int8: one code per byte)")
     ap.add_argument("--path", choices=["auto", "multi", "decode", "tc"], default="auto",
                     help="comparison case: force one of the library's layer paths (moe_layer_opts.path)")
     ap.add_argument("--int8-peak", action="store_true",
@@ -70,12 +72,16 @@ def parse(argv=None):
 
 
 def metric_for(wl, workload_id):
-    """The headline metric on its own workload; a labelled variant elsewhere."""
-    return METRIC if workload_id == 1 else f"MoE-layer tokens/s on {wl.name}; expert-weight HBM GB/s"
+    """The headline metric on its own workload, unmodified; a labelled variant
+    elsewhere."""
+    import workloads as W
+    if workload_id == 1 and wl.name == W.workload(1).name:
+        return METRIC
+    return f"MoE-layer tokens/s on {wl.name}; expert-weight HBM GB/s"
 
 
 def dtype_for(wl):
-    return "i8*i4->i32" if wl.wbits == 4 else "i8*i2->i32"
+    return f"i8*i{wl.wbits}->i32"
 
 
 def rank_token_sets(rank, n_sets):
@@ -723,7 +729,7 @@ def cache_arm(args, wl):
     line = {"metric": "MoE-layer decode tokens/s with an HBM expert cache (pool in pinned host memory)",
             "value": K * T / total, "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": Wm,
             "ms_per_step": 1e3 * total / K, "step_ms_median": 1e3 * statistics.median(wall),
-            "higher_is_better": True, "dtype": "i8*i4->i32" if wl.wbits == 4 else "i8*i2->i32",
+            "higher_is_better": True, "dtype": dtype_for(wl),
             "data": "synthetic", "config": {"workload": wl.name, "T": T, "experts": wl.n_experts,
                                             "top_k": wl.top_k, "cache_slots": args.cache_slots,
                                             "pool_gb": (wl.n_experts + wl.has_shared) * cfg.blob_bytes / 1e9},
@@ -790,6 +796,8 @@ def main(argv=None):
         wl = wl.replace(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
     if args.topp:
         wl = wl.replace(topp=args.topp, name=f"{wl.name}_topp{args.topp:g}")
+    if args.wbits and args.wbits != wl.wbits:
+        wl = wl.replace(wbits=args.wbits, name=f"{wl.name}_int{args.wbits}")
     if args.impl == "reference":
         reference_arm(args, wl)
     elif args.cache_slots:

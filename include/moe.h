@@ -5,7 +5,7 @@
  * of GLM-5.2 (744B): a DeepSeek-V3-style router picks top-k of E routed
  * experts per token (takumi3488 article, teacher-forcing section; top-8 of 256
  * in the coli info log), every expert is a feed-forward block whose weights are
- * packed int4 or int2 codes with per-row scales, dequantised on use and
+ * packed int4, int2 or int8 codes with per-row scales, dequantised on use and
  * multiplied against int8 activations with integer dot products (agentlenshq
  * summary, "Integer-Dot Kernels" and "Quantization"), and the routed outputs
  * are combined with the always-resident shared expert (agentlenshq summary,
@@ -34,7 +34,9 @@
  *    selection on score + bias, descending, ties to the lower expert index;
  *    weights = selected scores / their sum * routed_scale (bias not included).
  *  - codes: two's complement, low bits first (int4 byte = c0 | c1 << 4; int2
- *    byte = c0 | c1 << 2 | c2 << 4 | c3 << 6); int32 accumulation is exact.
+ *    byte = c0 | c1 << 2 | c2 << 4 | c3 << 6; int8: one code per byte, the
+ *    third width of the agentlenshq summary's "Quantization" item);
+ *    int32 accumulation is exact.
  *  - gate/up: g = acc_g * (s_row * s_x), u likewise, h = g / (1 + exp(-g)) * u
  *    (SwiGLU); h is requantised per (token, expert) with the activation rule.
  *  - down: y = acc_d * (s_row * s_h); out = sum_j w_j y_j + y_shared (fp32).
@@ -72,8 +74,8 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 /* Shape of one MoE layer.
  *  d: hidden size; f: expert intermediate size; n_experts: routed experts E;
  *  top_k: experts per token k; has_shared: 1 if a shared expert follows the E
- *  routed blobs; wbits: 4 or 2; routed_scale: factor on the renormalised
- *  routed weights (2.5 for GLM-5.2).
+ *  routed blobs; wbits: 4, 2 or 8 (codes per byte: 2, 4 or 1);
+ *  routed_scale: factor on the renormalised routed weights (2.5 for GLM-5.2).
  *  tc_min_tokens: calls of at least this many tokens run the experts on the
  *  int8 tensor-core (tcgen05) path (moe_layer with MOE_PATH_AUTO,
  *  moe_expert_ffn, moe_expert_down); 0 = library default (3: on B200 at the
