@@ -309,9 +309,11 @@ MOE_API moe_status moe_cache_init(const moe_config* cfg, moe_cache* cache, moe_s
 /* Makes every expert in idx (host int32 [T][top_k], -1 entries skipped)
  * resident: a hit refreshes the expert's use; a miss takes a free slot or
  * the least recently used slot whose expert this call does not select, and
- * issues one cudaMemcpyAsync of its blob on `stream`; then one copy of the
- * updated slot table.  MOE_ENOSPACE if n_slots cannot hold the call's
- * experts.  stats (nullable) receives this call's counts. */
+ * issues one cudaMemcpyAsync of its blob on `stream`; the changed slot_of
+ * entries are then written on `stream` by a small kernel whose (expert, slot)
+ * pairs travel as kernel arguments, so no host buffer outlives the call.
+ * MOE_ENOSPACE if n_slots cannot hold the call's experts.  stats (nullable)
+ * receives this call's counts. */
 MOE_API moe_status moe_cache_fetch(const moe_config* cfg, moe_cache* cache, const int32_t* idx, int32_t T,
                                    moe_stream_t stream, moe_cache_stats* stats);
 
