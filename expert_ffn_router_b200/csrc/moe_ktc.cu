@@ -7,6 +7,8 @@
 
 #include <algorithm>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "moe_launch.h"
 #include "moe_tc.cuh"
@@ -41,33 +43,57 @@ static cudaError_t make_pool_map(CUtensorMap* tm, const void* pool, uint64_t row
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Largest shared-memory footprint a CTA may take, and the slot count that
-// fills it; always large enough that one CTA occupies an SM (TMEM is
-// allocated whole).
-constexpr size_t kTcSmemBudget = 227 * 1024;
+// Shared memory of one CTA when `cps` CTAs share an SM (228 KB per SM, 1 KB
+// of it reserved per CTA), and the slot count that fills it.  Each CTA also
+// takes at least kTcSmemFloor[cps - 1], so that no more than `cps` CTAs fit
+// on an SM: their TMEM allocations (512 / cps columns) then always fit too.
+constexpr size_t kTcSmemBudget[2] = {227 * 1024, 113 * 1024};
+constexpr size_t kTcSmemFloor[2] = {120 * 1024, 78 * 1024};
 
-static int tc_slots(int nt_max, int wb) {
-    const size_t room = kTcSmemBudget - 1024 - sizeof(TcCtl);
+static int tc_slots(int nt_max, int wb, int cps) {
+    const size_t room = kTcSmemBudget[cps - 1] - 1024 - sizeof(TcCtl);
     return (int)std::min<size_t>(kTcMaxSlots, room / tc_slot_bytes(nt_max, wb));
 }
+
+// Two CTAs per SM where each one's half of TMEM still holds two A buffers
+// (int4 and int8 weights; an int2 chunk's A tiles take 128 columns).
+static int tc_cps(int wb) { return wb == 2 ? 1 : 2; }
 
 bool tc_shape_ok(const Dims& m) {
     // every assignment's token count fits the task split, and the slot ring
     // holds at least two chunks
-    return tc_slots(kTcNT, m.wb) >= 2 && m.d <= 8192 && m.f <= 8192;
+    return tc_slots(kTcNT, m.wb, tc_cps(m.wb)) >= 2 && m.d <= 8192 && m.f <= 8192;
 }
 
-template <int WB, int EPI>
+// Two CTAs per SM need the SM's whole shared memory as such (the carveout the
+// driver picks by default may leave room for one); set once per kernel and
+// device.  Without it the launch stays correct: the kernel's CTAs never wait
+// on one another, so CTAs that do not fit run after the first ones exit.
+static cudaError_t prefer_shared(const void* fn) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (done.count({dev, fn})) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) done.insert({dev, fn});
+    return e;
+}
+
+template <int WB, int EPI, int CPS>
 static cudaError_t launch_tc_t(const Params& p, const CUtensorMap& tm, int nt_max, cudaStream_t s) {
-    const int ns = tc_slots(nt_max, WB);
-    const size_t smem = std::max(tc_smem_bytes(ns, nt_max, WB), (size_t)120 * 1024);
-    auto fn = k_tc<WB, EPI>;
+    const int ns = tc_slots(nt_max, WB, CPS);
+    const size_t smem = std::max(tc_smem_bytes(ns, nt_max, WB), kTcSmemFloor[CPS - 1]);
+    auto fn = k_tc<WB, EPI, CPS>;
     cudaError_t e = allow_smem((const void*)fn, smem);
+    if (e == cudaSuccess && CPS > 1) e = prefer_shared((const void*)fn);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    fn<<<sms, kTcThreads, smem, s>>>(p, tm, ns, nt_max);
+    fn<<<CPS * sms, kTcThreads, smem, s>>>(p, tm, ns, nt_max);
     return cudaGetLastError();
 }
 
@@ -81,9 +107,9 @@ cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_
     else
         e = make_pool_map(&tm, p.pool, (uint64_t)p.m.f * wb / 8, (uint64_t)3 * p.m.d * E1);
     if (e != cudaSuccess) return e;
-    if (wb == 8) return stage == 0 ? launch_tc_t<8, 0>(p, tm, nt_max, s) : launch_tc_t<8, 1>(p, tm, nt_max, s);
-    if (wb == 4) return stage == 0 ? launch_tc_t<4, 0>(p, tm, nt_max, s) : launch_tc_t<4, 1>(p, tm, nt_max, s);
-    return stage == 0 ? launch_tc_t<2, 0>(p, tm, nt_max, s) : launch_tc_t<2, 1>(p, tm, nt_max, s);
+    if (wb == 8) return stage == 0 ? launch_tc_t<8, 0, 2>(p, tm, nt_max, s) : launch_tc_t<8, 1, 2>(p, tm, nt_max, s);
+    if (wb == 4) return stage == 0 ? launch_tc_t<4, 0, 2>(p, tm, nt_max, s) : launch_tc_t<4, 1, 2>(p, tm, nt_max, s);
+    return stage == 0 ? launch_tc_t<2, 0, 1>(p, tm, nt_max, s) : launch_tc_t<2, 1, 1>(p, tm, nt_max, s);
 }
 
 cudaError_t launch_tc_requant(const Params& p, cudaStream_t s) {

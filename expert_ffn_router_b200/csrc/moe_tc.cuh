@@ -41,9 +41,11 @@
 //  down    (EPI 1): rows [256 rb, 256 rb + 256) of d as two tiles; epilogue
 //                   y = acc (s_row s_h) to the per-assignment buffer (the
 //                   combine is a separate kernel) or straight to the output.
-// TMEM columns: two accumulator buffers [128 b, 128 b + 128) (tile 0 at
-// +0, tile 1 at +64, N <= 64), then the A buffers from column 256 (2 x KC/4
-// columns each: eight buffers for int8, four for int4, two for int2).  Every wait is bounded
+// TMEM columns (one CTA per SM): two accumulator buffers [128 b, 128 b + 128)
+// (tile 0 at +0, tile 1 at +64, N <= 64), then the A buffers from column 256
+// (2 x KC/4 columns each: eight buffers for int8, four for int4, two for
+// int2); two CTAs per SM (int4, int8): 256 columns each, one accumulator
+// buffer and A buffers from column 128 (four for int8, two for int4).  Every wait is bounded
 // (kWaitLimitNs); on a timeout the CTA records MOE_ETIMEOUT, lets its copies
 // and MMAs drain and exits.
 #pragma once
@@ -151,14 +153,23 @@ __device__ __forceinline__ size_t tc_b_offset(int kg, int j, int npad) {
     return ((size_t)kg * npad + j) * 16;
 }
 
-template <int WB, int EPI>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// CPS: CTAs per SM.  One CTA (CPS = 1) owns all 512 TMEM columns: two
+// accumulator buffers (the epilogue of a unit overlaps the next unit's MMAs)
+// and 256 columns of A buffers.  Two CTAs (CPS = 2) own 256 columns each: one
+// accumulator buffer and 128 columns of A buffers; the SM's tensor pipe then
+// interleaves the two CTAs' MMA streams, so neither CTA's serial waits
+// (slot, A buffer, accumulator hand-offs) leave it idle.
+template <int WB, int EPI, int CPS>
+__global__ void __launch_bounds__(kTcThreads, CPS)
     k_tc(const Params p, const __grid_constant__ CUtensorMap tmA, int ns, int nt_max) {
     constexpr int KC = tc_kc(WB);           // K columns per chunk
     constexpr int ACOLS = KC / 4;           // TMEM columns of one tile's A chunk
     constexpr int KSTEPS = KC / 32;
-    constexpr int NAB = 256 / (2 * ACOLS);  // TMEM A buffers
-    static_assert(NAB <= kTcMaxAB, "TcCtl holds kTcMaxAB A-buffer barriers");
+    constexpr uint32_t TCOLS = 512 / CPS;   // TMEM columns this CTA allocates
+    constexpr uint32_t NACC = 2 / CPS;      // accumulator buffers of 128 columns
+    constexpr uint32_t ABASE = 128 * NACC;  // first A-buffer column
+    constexpr int NAB = (int)(TCOLS - ABASE) / (2 * ACOLS);  // TMEM A buffers
+    static_assert(NAB >= 2 && NAB <= kTcMaxAB, "TcCtl holds kTcMaxAB A-buffer barriers; at least two keep unpack and MMA overlapped");
     constexpr int OFF = code_offset<WB>();
     extern __shared__ uint8_t tc_raw[];
     uint8_t* base = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023u)) & 1023u);
@@ -190,7 +201,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(&ctl->drain, 1);
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(&ctl->tmem_base, 512);
+    if (warp == 1) tmem_alloc(&ctl->tmem_base, TCOLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -253,9 +264,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int npad = tc_npad(idx_in(hdr, p.ws.tasks[ti].z, 1, kTcNT + 1, 644));
                 const uint32_t idesc = tc_idesc_u8s8(npad);
                 const uint32_t lbo = (uint32_t)npad * 16;
-                const uint32_t buf = uidx & 1u;
+                const uint32_t buf = uidx % NACC;
                 const uint32_t dcol = tbase + 128 * buf;
-                if (!tc_wait(&ctl->accempty[buf], ((uidx >> 1) & 1u) ^ 1u, hdr, 0x7103)) break;
+                if (!tc_wait(&ctl->accempty[buf], ((uidx / NACC) & 1u) ^ 1u, hdr, 0x7103)) break;
                 tc_fence_after();
                 for (int c = 0; c < nch; ++c) {
                     if (!tc_wait(&ctl->full[slot], ph, hdr, 0x7104) || !tc_wait(&ctl->afull[ab], abph, hdr, 0x7105)) {
@@ -264,7 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t bsm = smem_u32(base + (size_t)slot * slot_bytes + kTcSlotA);
-                    const uint32_t acol = tbase + 256 + ab * 2 * ACOLS;
+                    const uint32_t acol = tbase + ABASE + ab * 2 * ACOLS;
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
                         const uint64_t bdesc = smem_desc(bsm + ks * 2 * lbo, lbo, 128);
@@ -312,7 +323,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (ok) {
                     tc_fence_after();
                     const uint8_t* sp = base + (size_t)slot * slot_bytes;
-                    const uint32_t acol = tlane + 256 + ab * 2 * ACOLS + hh * (ACOLS / 2);
+                    const uint32_t acol = tlane + ABASE + ab * 2 * ACOLS + hh * (ACOLS / 2);
                     tc_unpack_tile<WB>(sp, row, hh, acol);
                     tc_unpack_tile<WB>(sp + kTcBox, row, hh, acol + ACOLS);
                     tmem_st_wait();
@@ -347,7 +358,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int4 task = p.ws.tasks[ti];
             const int n = idx_in(hdr, task.z, 1, kTcNT + 1, 645), npad = tc_npad(n);
             const int bx = idx_in(hdr, task.x, 0, p.m.E + p.m.has_shared, 648);
-            const uint32_t buf = uidx & 1u;
+            const uint32_t buf = uidx % NACC;
             named_sync(2, kTcEpi);  // the previous unit's metadata is no longer read
             if (etid < n) {
                 const int a = idx_in(hdr, p.ws.asg[idx_in(hdr, task.y + etid, 0, p.a_cap, 646)], 0, p.a_cap, 647);
@@ -362,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
             named_sync(2, kTcEpi);
-            if (ok) ok = tc_wait(&ctl->accfull[buf], (uidx >> 1) & 1u, hdr, 0x7109);
+            if (ok) ok = tc_wait(&ctl->accfull[buf], (uidx / NACC) & 1u, hdr, 0x7109);
             ok = __all_sync(kFull, ok);
             tc_fence_after();
             const uint32_t dcol = tlane + 128 * buf;
@@ -438,7 +449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        tmem_dealloc(tbase, 512);
+        tmem_dealloc(tbase, TCOLS);
     }
 }
 
