@@ -55,14 +55,13 @@ static int tc_slots(int nt_max, int wb, int cps) {
     return (int)std::min<size_t>(kTcMaxSlots, room / tc_slot_bytes(nt_max, wb));
 }
 
-// Two CTAs per SM where each one's half of TMEM still holds two A buffers
-// (int4 and int8 weights; an int2 chunk's A tiles take 128 columns).
-static int tc_cps(int wb) { return wb == 2 ? 1 : 2; }
+// CTAs per SM of the launches (k_tc's CPS).
+constexpr int kTcCps = 2;
 
 bool tc_shape_ok(const Dims& m) {
     // every assignment's token count fits the task split, and the slot ring
     // holds at least two chunks
-    return tc_slots(kTcNT, m.wb, tc_cps(m.wb)) >= 2 && m.d <= 8192 && m.f <= 8192;
+    return tc_slots(kTcNT, m.wb, kTcCps) >= 2 && m.d <= 8192 && m.f <= 8192;
 }
 
 // Two CTAs per SM need the SM's whole shared memory as such (the carveout the
@@ -107,9 +106,10 @@ cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_
     else
         e = make_pool_map(&tm, p.pool, (uint64_t)p.m.f * wb / 8, (uint64_t)3 * p.m.d * E1);
     if (e != cudaSuccess) return e;
-    if (wb == 8) return stage == 0 ? launch_tc_t<8, 0, 2>(p, tm, nt_max, s) : launch_tc_t<8, 1, 2>(p, tm, nt_max, s);
-    if (wb == 4) return stage == 0 ? launch_tc_t<4, 0, 2>(p, tm, nt_max, s) : launch_tc_t<4, 1, 2>(p, tm, nt_max, s);
-    return stage == 0 ? launch_tc_t<2, 0, 1>(p, tm, nt_max, s) : launch_tc_t<2, 1, 1>(p, tm, nt_max, s);
+    constexpr int C = kTcCps;
+    if (wb == 8) return stage == 0 ? launch_tc_t<8, 0, C>(p, tm, nt_max, s) : launch_tc_t<8, 1, C>(p, tm, nt_max, s);
+    if (wb == 4) return stage == 0 ? launch_tc_t<4, 0, C>(p, tm, nt_max, s) : launch_tc_t<4, 1, C>(p, tm, nt_max, s);
+    return stage == 0 ? launch_tc_t<2, 0, C>(p, tm, nt_max, s) : launch_tc_t<2, 1, C>(p, tm, nt_max, s);
 }
 
 cudaError_t launch_tc_requant(const Params& p, cudaStream_t s) {

@@ -9,7 +9,8 @@
 //  A  weight codes.  A TMA box of 128 rows x 64 packed bytes (64-byte swizzle)
 //     lands in shared memory; the unpack warps split each 32-bit word into
 //     offset-binary bytes (u = c + 8 for int4, c + 2 for int2, the same masks
-//     as the dp4a kernels) and store them to TMEM, from where the MMA reads A.
+//     as the dp4a kernels; int8 bytes with the sign bit flipped, c + 128) and
+//     store them to TMEM, from where the MMA reads A.
 //     Unsigned A times signed activations gives sum(u x) = sum(c x) + off sum(x);
 //     the epilogue subtracts off * sum(x).
 //  B  int8 activations (or requantised h) of the task's tokens, in the
@@ -19,10 +20,13 @@
 //     writes it per task and K chunk, so one bulk copy brings a chunk's B into
 //     shared memory.
 //
-// An M = 128, K = 32 MMA costs a fixed ~90 SM cycles for any N <= 128, so one
-// 128-row tile streams at most ~2 packed bytes per cycle per tile; the kernel
-// keeps the MMA pipe issuing back to back.  Persistent, one CTA per SM,
-// 448 threads:
+// An M = 128, K = 32 MMA issued back to back takes ~97 SM cycles for any
+// N <= 128 when each one accumulates into the previous one's tile, ~54 when
+// two tiles alternate (as here), ~68 with two commits per eight MMAs
+// (microbenchmark on B200), while an SM's share of HBM bandwidth delivers
+// one int4 A step (2 KB of packed codes) in ~90 cycles: the MMA stream keeps
+// up with HBM only while it does not stall.  Persistent, two CTAs per SM (their
+// MMA streams interleave on the SM's tensor pipe), 448 threads each:
 //  warp 0      TMA producer: per K chunk two A boxes + the B chunk into a
 //              ring of shared-memory slots (full / empty mbarriers);
 //  warp 1      TMEM allocator and MMA issuer (one thread): per chunk
@@ -41,11 +45,11 @@
 //  down    (EPI 1): rows [256 rb, 256 rb + 256) of d as two tiles; epilogue
 //                   y = acc (s_row s_h) to the per-assignment buffer (the
 //                   combine is a separate kernel) or straight to the output.
-// TMEM columns (one CTA per SM): two accumulator buffers [128 b, 128 b + 128)
+// TMEM columns (CPS = 1, one CTA per SM): two accumulator buffers [128 b, 128 b + 128)
 // (tile 0 at +0, tile 1 at +64, N <= 64), then the A buffers from column 256
 // (2 x KC/4 columns each: eight buffers for int8, four for int4, two for
-// int2); two CTAs per SM (int4, int8): 256 columns each, one accumulator
-// buffer and A buffers from column 128 (four for int8, two for int4).  Every wait is bounded
+// int2); two CTAs per SM: 256 columns each, one accumulator buffer and A
+// buffers from column 128 (four for int8, two for int4, one for int2).  Every wait is bounded
 // (kWaitLimitNs); on a timeout the CTA records MOE_ETIMEOUT, lets its copies
 // and MMAs drain and exits.
 #pragma once
@@ -155,10 +159,14 @@ __device__ __forceinline__ size_t tc_b_offset(int kg, int j, int npad) {
 
 // CPS: CTAs per SM.  One CTA (CPS = 1) owns all 512 TMEM columns: two
 // accumulator buffers (the epilogue of a unit overlaps the next unit's MMAs)
-// and 256 columns of A buffers.  Two CTAs (CPS = 2) own 256 columns each: one
-// accumulator buffer and 128 columns of A buffers; the SM's tensor pipe then
-// interleaves the two CTAs' MMA streams, so neither CTA's serial waits
-// (slot, A buffer, accumulator hand-offs) leave it idle.
+// and 256 columns of A buffers.  Two CTAs (CPS = 2, what the library
+// launches) own 256 columns each: one accumulator buffer and 128 columns of
+// A buffers (one for int2); the SM's tensor pipe then interleaves the two
+// CTAs' MMA streams, so neither CTA's serial waits (slot, A buffer,
+// accumulator hand-offs) leave it idle.  Measured on B200, two CTAs beat one
+// for every width: at T = 512 (int4) the gate/up kernel takes 505 us instead
+// of 611, on the int2 stack 156 us instead of 167, although an int2 CTA then
+// unpacks a chunk only after the previous one's MMAs have completed.
 template <int WB, int EPI, int CPS>
 __global__ void __launch_bounds__(kTcThreads, CPS)
     k_tc(const Params p, const __grid_constant__ CUtensorMap tmA, int ns, int nt_max) {
@@ -169,7 +177,7 @@ __global__ void __launch_bounds__(kTcThreads, CPS)
     constexpr uint32_t NACC = 2 / CPS;      // accumulator buffers of 128 columns
     constexpr uint32_t ABASE = 128 * NACC;  // first A-buffer column
     constexpr int NAB = (int)(TCOLS - ABASE) / (2 * ACOLS);  // TMEM A buffers
-    static_assert(NAB >= 2 && NAB <= kTcMaxAB, "TcCtl holds kTcMaxAB A-buffer barriers; at least two keep unpack and MMA overlapped");
+    static_assert(NAB >= 1 && NAB <= kTcMaxAB, "TcCtl holds kTcMaxAB A-buffer barriers");
     constexpr int OFF = code_offset<WB>();
     extern __shared__ uint8_t tc_raw[];
     uint8_t* base = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023u)) & 1023u);
