@@ -29,16 +29,20 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D uint8 view of the pool: `rows` rows of `rowbytes` bytes; box of
-// 64 bytes x 128 rows, 64-byte swizzle, zero fill outside the tensor.
-static cudaError_t make_pool_map(CUtensorMap* tm, const void* pool, uint64_t rowbytes, uint64_t rows) {
+// tc_box_w(wb, stage) bytes x 128 rows with the swizzle of that width (64 or
+// 128 bytes), zero fill outside the tensor.
+static cudaError_t make_pool_map(CUtensorMap* tm, const void* pool, uint64_t rowbytes, uint64_t rows, int wb,
+                                 int stage) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {rowbytes, rows};
     const cuuint64_t strides[1] = {rowbytes};
-    const cuuint32_t box[2] = {64, 128};
+    const int bw = tc_box_w(wb, stage);
+    const cuuint32_t box[2] = {(cuuint32_t)bw, 128};
     const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw = bw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pool), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -50,9 +54,9 @@ static cudaError_t make_pool_map(CUtensorMap* tm, const void* pool, uint64_t row
 constexpr size_t kTcSmemBudget[2] = {227 * 1024, 113 * 1024};
 constexpr size_t kTcSmemFloor[2] = {120 * 1024, 78 * 1024};
 
-static int tc_slots(int nt_max, int wb, int cps) {
+static int tc_slots(int nt_max, int wb, int cps, int epi) {
     const size_t room = kTcSmemBudget[cps - 1] - 1024 - sizeof(TcCtl);
-    return (int)std::min<size_t>(kTcMaxSlots, room / tc_slot_bytes(nt_max, wb));
+    return (int)std::min<size_t>(kTcMaxSlots, room / tc_slot_bytes(nt_max, wb, epi));
 }
 
 // CTAs per SM of the launches (k_tc's CPS).
@@ -61,7 +65,8 @@ constexpr int kTcCps = 2;
 bool tc_shape_ok(const Dims& m) {
     // every assignment's token count fits the task split, and the slot ring
     // holds at least two chunks
-    return tc_slots(kTcNT, m.wb, kTcCps) >= 2 && m.d <= 8192 && m.f <= 8192;
+    return tc_slots(kTcNT, m.wb, kTcCps, 0) >= 2 && tc_slots(kTcNT, m.wb, kTcCps, 1) >= 2 && m.d <= 8192 &&
+           m.f <= 8192;
 }
 
 // Two CTAs per SM need the SM's whole shared memory as such (the carveout the
@@ -83,8 +88,8 @@ static cudaError_t prefer_shared(const void* fn) {
 
 template <int WB, int EPI, int CPS>
 static cudaError_t launch_tc_t(const Params& p, const CUtensorMap& tm, int nt_max, cudaStream_t s) {
-    const int ns = tc_slots(nt_max, WB, CPS);
-    const size_t smem = std::max(tc_smem_bytes(ns, nt_max, WB), kTcSmemFloor[CPS - 1]);
+    const int ns = tc_slots(nt_max, WB, CPS, EPI);
+    const size_t smem = std::max(tc_smem_bytes(ns, nt_max, WB, EPI), kTcSmemFloor[CPS - 1]);
     auto fn = k_tc<WB, EPI, CPS>;
     cudaError_t e = allow_smem((const void*)fn, smem);
     if (e == cudaSuccess && CPS > 1) e = prefer_shared((const void*)fn);
@@ -102,9 +107,9 @@ cudaError_t launch_tc_expert(const Params& p, int stage, int nt_max, cudaStream_
     const int wb = p.m.wb;
     cudaError_t e;
     if (stage == 0)
-        e = make_pool_map(&tm, p.pool, (uint64_t)p.m.d * wb / 8, (uint64_t)3 * p.m.f * E1);
+        e = make_pool_map(&tm, p.pool, (uint64_t)p.m.d * wb / 8, (uint64_t)3 * p.m.f * E1, wb, 0);
     else
-        e = make_pool_map(&tm, p.pool, (uint64_t)p.m.f * wb / 8, (uint64_t)3 * p.m.d * E1);
+        e = make_pool_map(&tm, p.pool, (uint64_t)p.m.f * wb / 8, (uint64_t)3 * p.m.d * E1, wb, 1);
     if (e != cudaSuccess) return e;
     constexpr int C = kTcCps;
     if (wb == 8) return stage == 0 ? launch_tc_t<8, 0, C>(p, tm, nt_max, s) : launch_tc_t<8, 1, C>(p, tm, nt_max, s);

@@ -64,8 +64,20 @@ constexpr int kTcThreads = 448;
 constexpr int kTcUnpack = 256;                 // warps 2-9
 constexpr int kTcEpiWarp0 = 10;                // warps 10-13
 constexpr int kTcEpi = 128;
-constexpr int kTcBox = 128 * 64;               // one A box: 128 rows x 64 packed bytes
-constexpr int kTcSlotA = 2 * kTcBox;           // both tiles of a chunk
+// A weight box: 128 rows x tc_box_w bytes of packed codes, one box per tile
+// per ring slot.  Rows loaded 128 bytes (two chunks of 64 bytes) at a time
+// with the 128-byte swizzle arrive whole instead of through promoted L2 lines
+// that may be evicted before their chunk is loaded, but a slot is then
+// released only after both chunks.  Measured on B200 (two CTAs per SM): the
+// down kernels and int8 weights gain (T = 512, int4 down: 285 us instead of
+// 307; int8 gate/up at T = 8: 264 instead of 270), the int4 gate/up kernel
+// loses (519 instead of 506), so it keeps 64-byte boxes, as does int2, whose
+// operand-B chunks are four times larger (two-chunk slots would not fit
+// twice in a CTA's shared memory).
+__host__ __device__ constexpr int tc_box_w(int wb, int epi) { return wb == 2 || (wb == 4 && epi == 0) ? 64 : 128; }
+__host__ __device__ constexpr int tc_cpl(int wb, int epi) { return tc_box_w(wb, epi) / 64; }  // chunks per slot
+__host__ __device__ constexpr int tc_box_bytes(int wb, int epi) { return 128 * tc_box_w(wb, epi); }
+__host__ __device__ constexpr int tc_slot_a(int wb, int epi) { return 2 * tc_box_bytes(wb, epi); }  // both tiles
 constexpr int kTcMaxSlots = 8;
 constexpr int kTcMaxAB = 8;                    // TMEM A buffers: 256 columns / (2 tiles x KC/4), KC = 64 for int8
 
@@ -79,11 +91,11 @@ struct TcCtl {
     int cs[kTcNT];
 };
 
-__host__ __device__ constexpr int tc_slot_bytes(int nt_max, int wb) {
-    return (kTcSlotA + nt_max * tc_kc(wb) + 1023) / 1024 * 1024;
+__host__ __device__ constexpr int tc_slot_bytes(int nt_max, int wb, int epi) {
+    return (tc_slot_a(wb, epi) + tc_cpl(wb, epi) * nt_max * tc_kc(wb) + 1023) / 1024 * 1024;
 }
-__host__ __device__ constexpr size_t tc_smem_bytes(int ns, int nt_max, int wb) {
-    return 1024 + (size_t)ns * tc_slot_bytes(nt_max, wb) + sizeof(TcCtl);
+__host__ __device__ constexpr size_t tc_smem_bytes(int ns, int nt_max, int wb, int epi) {
+    return 1024 + (size_t)ns * tc_slot_bytes(nt_max, wb, epi) + sizeof(TcCtl);
 }
 
 // Same as mbar_wait_bounded, but also gives up when another wait of the call
@@ -104,17 +116,23 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, WsHeader
 }
 
 // Unpack one thread's share of one A tile of a chunk into TMEM.  Row `row` of
-// the box (64 packed bytes, 64-byte swizzle: 16-byte unit j of row r sits at
-// unit j ^ ((r >> 1) & 3)); half `hh` takes units 2hh and 2hh+1.
-template <int WB>
-__device__ __forceinline__ void tc_unpack_tile(const uint8_t* box, int row, int hh, uint32_t taddr) {
-    const uint8_t* rp = box + row * 64;
-    const int sw = (row >> 1) & 3;
+// the box: BW packed bytes, 64-byte rows with the 64-byte swizzle
+// (16-byte unit j of row r at unit j ^ ((r >> 1) & 3)) or 128-byte rows with
+// the 128-byte swizzle (unit j at j ^ (r & 7)); the chunk is half `hc` of a
+// 128-byte row (units 4hc .. 4hc + 3), and half `hh` of the chunk takes its
+// units 2hh and 2hh+1.
+template <int BW>
+__device__ __forceinline__ int tc_unit(int row, int hc, int u) {
+    return BW == 64 ? u ^ ((row >> 1) & 3) : (4 * hc + u) ^ (row & 7);
+}
+template <int WB, int BW>
+__device__ __forceinline__ void tc_unpack_tile(const uint8_t* box, int row, int hh, int hc, uint32_t taddr) {
+    const uint8_t* rp = box + row * BW;
     if (WB == 8) {  // one code per byte: flip each sign bit
         uint32_t w[8];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rp + (((2 * hh + j) ^ sw) << 4));
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + (tc_unit<BW>(row, hc, 2 * hh + j) << 4));
             w[4 * j] = v.x ^ 0x80808080u;
             w[4 * j + 1] = v.y ^ 0x80808080u;
             w[4 * j + 2] = v.z ^ 0x80808080u;
@@ -125,7 +143,7 @@ __device__ __forceinline__ void tc_unpack_tile(const uint8_t* box, int row, int 
         uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rp + (((2 * hh + j) ^ sw) << 4));
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + (tc_unit<BW>(row, hc, 2 * hh + j) << 4));
             const uint32_t in[4] = {v.x ^ 0x88888888u, v.y ^ 0x88888888u, v.z ^ 0x88888888u, v.w ^ 0x88888888u};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -138,7 +156,7 @@ __device__ __forceinline__ void tc_unpack_tile(const uint8_t* box, int row, int 
         uint32_t w[32];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rp + (((2 * hh + j) ^ sw) << 4));
+            const uint4 v = *reinterpret_cast<const uint4*>(rp + (tc_unit<BW>(row, hc, 2 * hh + j) << 4));
             const uint32_t in[4] = {v.x ^ 0xAAAAAAAAu, v.y ^ 0xAAAAAAAAu, v.z ^ 0xAAAAAAAAu, v.w ^ 0xAAAAAAAAu};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -179,9 +197,11 @@ __global__ void __launch_bounds__(kTcThreads, CPS)
     constexpr int NAB = (int)(TCOLS - ABASE) / (2 * ACOLS);  // TMEM A buffers
     static_assert(NAB >= 1 && NAB <= kTcMaxAB, "TcCtl holds kTcMaxAB A-buffer barriers");
     constexpr int OFF = code_offset<WB>();
+    constexpr int BW = tc_box_w(WB, EPI), CPL = tc_cpl(WB, EPI), BOX = tc_box_bytes(WB, EPI);
+    constexpr int SLOT_A = tc_slot_a(WB, EPI);
     extern __shared__ uint8_t tc_raw[];
     uint8_t* base = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023u)) & 1023u);
-    const int slot_bytes = tc_slot_bytes(nt_max, WB);
+    const int slot_bytes = tc_slot_bytes(nt_max, WB, EPI);
     TcCtl* ctl = reinterpret_cast<TcCtl*>(base + (size_t)ns * slot_bytes);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     WsHeader* hdr = p.ws.hdr;
@@ -238,16 +258,19 @@ __global__ void __launch_bounds__(kTcThreads, CPS)
                 }
                 const uint8_t* bsrc =
                     bbuf + (size_t)idx_in(hdr, task.w, 0, (int)tc_rows_bound(p.m) - npad + 1, 643) * kpad;
-                for (int c = 0; c < nch; ++c) {
+                // one slot per CPL chunks (the unit's last slot may hold
+                // fewer): both tiles' boxes and the chunks' operand B
+                for (int c = 0; c < nch; c += CPL) {
                     if (!tc_wait(&ctl->empty[slot], ph ^ 1u, hdr, 0x7101)) {
                         ok = false;
                         break;
                     }
+                    const uint32_t nc = (uint32_t)min(CPL, nch - c);
                     uint8_t* sp = base + (size_t)slot * slot_bytes;
-                    mbar_arrive_expect_tx(&ctl->full[slot], kTcSlotA + bbytes);
+                    mbar_arrive_expect_tx(&ctl->full[slot], SLOT_A + nc * bbytes);
                     tma_load_2d(sp, &tmA, c * 64, y0, &ctl->full[slot], pol);
-                    tma_load_2d(sp + kTcBox, &tmA, c * 64, y1, &ctl->full[slot], pol);
-                    bulk_g2s(sp + kTcSlotA, bsrc + (size_t)c * bbytes, bbytes, &ctl->full[slot]);
+                    tma_load_2d(sp + BOX, &tmA, c * 64, y1, &ctl->full[slot], pol);
+                    bulk_g2s(sp + SLOT_A, bsrc + (size_t)c * bbytes, nc * bbytes, &ctl->full[slot]);
                     ++issued;
                     if (++slot == ns) {
                         slot = 0;
@@ -282,7 +305,8 @@ __global__ void __launch_bounds__(kTcThreads, CPS)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t bsm = smem_u32(base + (size_t)slot * slot_bytes + kTcSlotA);
+                    const int hc = c % CPL;  // which chunk of the slot
+                    const uint32_t bsm = smem_u32(base + (size_t)slot * slot_bytes + SLOT_A) + hc * npad * KC;
                     const uint32_t acol = tbase + ABASE + ab * 2 * ACOLS;
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
@@ -292,12 +316,14 @@ __global__ void __launch_bounds__(kTcThreads, CPS)
                         tc_mma_i8_ts(dcol + 64, acol + ACOLS + ks * 8, bdesc, idesc, acc);
                     }
                     issued = true;
-                    tc_commit(&ctl->empty[slot]);
-                    tc_commit(&ctl->afree[ab]);
-                    if (++slot == ns) {
-                        slot = 0;
-                        ph ^= 1u;
+                    if (hc == CPL - 1 || c == nch - 1) {  // the slot's last chunk
+                        tc_commit(&ctl->empty[slot]);
+                        if (++slot == ns) {
+                            slot = 0;
+                            ph ^= 1u;
+                        }
                     }
+                    tc_commit(&ctl->afree[ab]);
                     if (++ab == NAB) {
                         ab = 0;
                         abph ^= 1u;
@@ -326,26 +352,29 @@ __global__ void __launch_bounds__(kTcThreads, CPS)
         bool ok = true;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
             for (int c = 0; c < nch; ++c) {
+                const int hc = c % CPL;  // which chunk of the slot
                 if (ok) ok = tc_wait(&ctl->full[slot], ph, hdr, 0x7107) && tc_wait(&ctl->afree[ab], abph ^ 1u, hdr, 0x7108);
                 ok = __all_sync(kFull, ok);
                 if (ok) {
                     tc_fence_after();
                     const uint8_t* sp = base + (size_t)slot * slot_bytes;
                     const uint32_t acol = tlane + ABASE + ab * 2 * ACOLS + hh * (ACOLS / 2);
-                    tc_unpack_tile<WB>(sp, row, hh, acol);
-                    tc_unpack_tile<WB>(sp + kTcBox, row, hh, acol + ACOLS);
+                    tc_unpack_tile<WB, BW>(sp, row, hh, hc, acol);
+                    tc_unpack_tile<WB, BW>(sp + BOX, row, hh, hc, acol + ACOLS);
                     tmem_st_wait();
                 }
                 // this warp's reads of the slot (generic proxy) before the
                 // producer's next TMA load into it (async proxy), which the
-                // MMA's commit of this chunk lets it issue
+                // MMA's commit of the slot's last chunk lets it issue
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->afull[ab]);
-                if (++slot == ns) {
-                    slot = 0;
-                    ph ^= 1u;
+                if (hc == CPL - 1 || c == nch - 1) {  // the slot's last chunk
+                    if (++slot == ns) {
+                        slot = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (++ab == NAB) {
                     ab = 0;
