@@ -273,6 +273,15 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                  "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+// The same with an L2 cache policy (e.g. evict-first for bytes read once).
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
 // TOPK/TOPP truncation of one warp's k selected slots (lane j holds slot j).
 // With 0 < topp < 1, slot j is kept iff j == 0 or cex -- the float sum of the
 // scores of slots 0..j-1, added in slot order -- is below fl(topp * ssum),
