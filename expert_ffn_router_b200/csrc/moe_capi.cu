@@ -258,10 +258,12 @@ static cudaError_t launch_router(Params& p, const XT* x, int do_quant, int bucke
         k_quantize<XT><<<std::min(T, 65535), kThreads, 0, s>>>(x, T, d, p.ws.xq, p.ws.sx, p.ws.xcs);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    // split d so that the tiled GEMM fills the GPU (slices of whole 32-column steps)
+    // split d so that the tiled GEMM puts about four CTAs on each of the 148
+    // SMs (slices of whole 32-column steps; measured on B200 at T = 512 and
+    // 8192: four per SM beat two by ~10% of the router's time, eight lose)
     const int tiles = ((E + 63) / 64) * ((T + 63) / 64);
     const int ksteps = d / 32;
-    int ks = std::max(1, std::min(std::min(ksteps, kRouterKsplitMax), (2 * 148 + tiles - 1) / tiles));
+    int ks = std::max(1, std::min(std::min(ksteps, kRouterKsplitMax), (4 * 148 + tiles - 1) / tiles));
     const int per = (ksteps + ks - 1) / ks;
     ks = (ksteps + per - 1) / per;
     p.ksplit = ks;
