@@ -490,6 +490,32 @@ __global__ void __launch_bounds__(kTcThreads, CPS)
     }
 }
 
+// The task whose padded rows hold row R (tasks are in row order, task.w
+// ascending): a binary search over the tasks' first rows, in shared memory
+// when the CTA has staged them (tw_s), else in global memory.  Staging turns
+// the search's dependent global loads (several L2 round trips per row) into
+// one coalesced load per CTA.
+constexpr int kTcTaskCache = 2048;
+__device__ __forceinline__ int tc_task_of_row(const Params& p, const int* tw_s, int n_tasks, int R) {
+    int lo = 0, hi = n_tasks - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const int w = tw_s ? tw_s[mid] : __ldg(&p.ws.tasks[mid].w);
+        if (w <= R) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+// Stages the tasks' first rows in shared memory if they fit (all threads of
+// the CTA call it); returns the staged array or nullptr.
+__device__ __forceinline__ const int* tc_stage_task_rows(const Params& p, int* tw_s, int n_tasks) {
+    const bool cached = n_tasks <= kTcTaskCache;
+    if (cached)
+        for (int i = threadIdx.x; i < n_tasks; i += blockDim.x) tw_s[i] = __ldg(&p.ws.tasks[i].w);
+    __syncthreads();
+    return cached ? tw_s : nullptr;
+}
+
 // a4's input rule on the tensor-core path: requantise each assignment's h
 // (max |h| from the gate/up epilogue) into the down operand B, in the MMA
 // layout, with its scale and code sum; leaves the maxima zeroed.  One warp per
@@ -500,13 +526,10 @@ __global__ void __launch_bounds__(kThreads) k_tc_requant(const Params p) {
     const int f = p.m.f;
     const int n_tasks = p.ws.hdr->n_tasks, rows = p.ws.hdr->tc_rows;
     const int kpad = tc_kpad(f, WB), npk = kpad / 16;
+    __shared__ int tw_s[kTcTaskCache];
+    const int* tw = tc_stage_task_rows(p, tw_s, n_tasks);
     for (int R = blockIdx.x * kWarps + warp; R < rows; R += gridDim.x * kWarps) {
-        int lo = 0, hi = n_tasks - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(&p.ws.tasks[mid].w) <= R) lo = mid;
-            else hi = mid - 1;
-        }
+        const int lo = tc_task_of_row(p, tw, n_tasks, R);
         const int4 task = __ldg(p.ws.tasks + lo);
         const int j = idx_in(p.ws.hdr, R - task.w, 0, kTcNT + 16, 651), npad = tc_npad(task.z);
         const bool live = j < task.z;
@@ -560,13 +583,10 @@ __global__ void __launch_bounds__(kThreads) k_tc_gather(const Params p, const in
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tasks = p.ws.hdr->n_tasks, rows = p.ws.hdr->tc_rows;
     const int npk = kpad / 16;
+    __shared__ int tw_s[kTcTaskCache];
+    const int* tw = tc_stage_task_rows(p, tw_s, n_tasks);
     for (int R = blockIdx.x * kWarps + warp; R < rows; R += gridDim.x * kWarps) {
-        int lo = 0, hi = n_tasks - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(&p.ws.tasks[mid].w) <= R) lo = mid;
-            else hi = mid - 1;
-        }
+        const int lo = tc_task_of_row(p, tw, n_tasks, R);
         const int4 task = __ldg(p.ws.tasks + lo);
         const int j = idx_in(p.ws.hdr, R - task.w, 0, kTcNT + 16, 654), npad = tc_npad(task.z);
         const int key = j < task.z ? idx_in(p.ws.hdr, __ldg(p.ws.asg + idx_in(p.ws.hdr, task.y + j, 0, p.a_cap, 655)),
