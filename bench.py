@@ -797,7 +797,9 @@ def main(argv=None):
     if args.topp:
         wl = wl.replace(topp=args.topp, name=f"{wl.name}_topp{args.topp:g}")
     if args.wbits and args.wbits != wl.wbits:
-        wl = wl.replace(wbits=args.wbits, name=f"{wl.name}_int{args.wbits}")
+        tag, new = f"_int{wl.wbits}", f"_int{args.wbits}"
+        name = wl.name.replace(tag, new) if tag in wl.name else wl.name + new
+        wl = wl.replace(wbits=args.wbits, name=name)
     if args.impl == "reference":
         reference_arm(args, wl)
     elif args.cache_slots:

@@ -59,6 +59,24 @@ def test_labels():
     assert bench.metric_for(W.workload(3), 3) != bench.METRIC
     assert bench.dtype_for(W.workload(1)) == "i8*i4->i32"
     assert bench.dtype_for(W.workload(4)) == "i8*i2->i32"
+    # a modified headline workload (int8 codes, truncation, more tokens) is
+    # a labelled variant, not the headline metric
+    int8 = W.workload(1).replace(wbits=8, name=W.workload(1).name + "_int8")
+    assert bench.dtype_for(int8) == "i8*i8->i32"
+    assert bench.metric_for(int8, 1) != bench.METRIC and int8.name in bench.metric_for(int8, 1)
+    topp = W.workload(1).replace(topp=0.7, name=W.workload(1).name + "_topp0.7")
+    assert bench.metric_for(topp, 1) != bench.METRIC
+
+
+def test_variant_options_name_the_workload(monkeypatch):
+    seen = {}
+    monkeypatch.setattr(bench, "gpu_arm", lambda args, wl: seen.update(wl=wl))
+    bench.main(["--wbits", "8", "--tokens", "8", "--topp", "0.7"])
+    wl = seen["wl"]
+    assert (wl.wbits, wl.T, wl.topp) == (8, 8, 0.7)
+    assert wl.name == "decode_T1_d6144_f2048_e256_k8_int8_T8_topp0.7"
+    bench.main(["--wbits", "4"])  # the workload's own width: unchanged
+    assert seen["wl"] == W.workload(1)
 
 
 def test_rank_token_streams():
