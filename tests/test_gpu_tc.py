@@ -144,6 +144,33 @@ def test_tc_layer_prefill_sampled_matches_multi():
     print("prefill tensor-core sampled rel L2:", err)
 
 
+def test_tc_layer_hot_experts_split_tasks():
+    """Skewed routing at T = 512 (the int2 workload's Zipf-biased router, one
+    layer): the most-loaded experts receive well over 64 tokens, so their
+    assignments are cut into several tensor-core tasks and their weights are
+    read once per task.  The tokens of the hottest expert on both sides of
+    each task boundary, and its first and last, against the oracle; every
+    token against the dp4a multi-kernel layer."""
+    wl = W.workload(4).replace(name="skewed_int2_T512", T=512, n_layers=1)
+    L = W.layer(wl, 0, 0)
+    dl = W.device_layer(wl, 0, 0, host=L)
+    x = x_host(wl, 3, wl.T)
+    out, g_idx, _ = run_layer_tc(wl, dl, x)
+    counts = np.bincount(g_idx[g_idx >= 0].ravel(), minlength=wl.n_experts)
+    hot = int(counts.argmax())
+    assert counts[hot] > 2 * 64, counts[hot]  # at least three tasks
+    hot_tokens = np.nonzero((g_idx == hot).any(axis=1))[0]  # (token, slot) order = task order
+    picks = {0, len(hot_tokens) - 1}
+    for b in range(64, len(hot_tokens), 64):
+        picks |= {b - 1, b}
+    tokens = sorted({int(hot_tokens[i]) for i in picks})
+    err, _ = compare_layer(wl, L, x, out, g_idx, tokens)
+    out_m, idx_m, _ = run_layer_tc(wl, dl, x, path=M.MOE_PATH_MULTI)
+    np.testing.assert_array_equal(g_idx, idx_m)
+    assert rel_l2(out.cpu().numpy(), out_m.cpu().numpy()) <= 1e-3
+    print(f"hottest expert {hot}: {counts[hot]} tokens, {len(tokens)} sampled, rel L2 {err:.3g}")
+
+
 def test_tc_workspace_reuse_deterministic():
     """Calls of different T alternating the tensor-core and decode paths on one
     workspace: counters self-reset, results identical call to call."""
