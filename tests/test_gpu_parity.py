@@ -329,7 +329,7 @@ def run_stack(wl, n_layers, token_subset):
     return resid.cpu().numpy()[token_subset], idxs, r
 
 
-@pytest.mark.parametrize("which,n_layers,tokens", [(2, 8, [0, 1, 2, 3]), (4, 24, [0, 37])])
+@pytest.mark.parametrize("which,n_layers,tokens", [(2, 8, [0, 1, 2, 3]), (4, 24, [0, 21, 37, 63])])
 def test_stacked_layers(which, n_layers, tokens):
     wl = W.workload(which)
     g_x, g_idxs, r = run_stack(wl, n_layers, tokens)
